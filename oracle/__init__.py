@@ -1,0 +1,35 @@
+"""CPU oracle for the sparse-attention selection step.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports, calls or links
+this package: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` (and its ``--impl reference`` arm) may use it.  It shares no
+code with the CUDA library under ``sparse_attention_top_ds_b200/csrc``.
+
+Everything here is a plain, slow, single-threaded restatement of what the
+selection step computes, in float64:
+
+* ``encoding``   -- IEEE binary32 / bfloat16 bit patterns decoded to float64.
+* ``topk``       -- row-wise top-k of given scores: a stable descending sort,
+                    ties to the lower index (DeepSelect hub page, the two
+                    use-case paragraphs: lightning indexer at topk=512 in
+                    bfloat16, sampling over a ~128K vocabulary in float32, and
+                    the ``sorted_index`` / ``return_value`` options).
+* ``indexer``    -- the lightning-indexer score
+                    ``score[t,s] = sum_h w[t,h] * max(0, q[t,h,:] . k[s,:])``
+                    (NKI pull request "Add DeepSeek-V4 CSA attention kernels",
+                    "How the algorithm works", steps table, row 2) followed by
+                    the same top-k.
+
+Every function is pinned by the ``-m "not gpu"`` tests in ``tests/test_oracle_*``
+against brute force, closed forms, hand-worked examples under ``tests/golden``
+and invariants; no function here is "parity unpinned".
+"""
+
+from .encoding import decode_bf16, decode_f32, NEG_INF_BF16, NEG_INF_F32
+from .topk import topk_rows, topk_row
+from .indexer import indexer_scores, indexer_topk
+
+__all__ = [
+    "decode_bf16", "decode_f32", "NEG_INF_BF16", "NEG_INF_F32",
+    "topk_rows", "topk_row", "indexer_scores", "indexer_topk",
+]
