@@ -1,0 +1,158 @@
+/*
+ * ds_topk.h -- C ABI of libdstopk.so, the selection step of DeepSeek-style
+ * sparse attention on B200 (sm_100a).
+ *
+ * Two operations, as described on the pages this library follows:
+ *
+ *  - Row-wise top-k of given scores (DeepSelect hub page, use-case paragraphs:
+ *    pick the top-k positions of every score row; bfloat16 rows for the
+ *    lightning indexer, float32 rows over a ~129K vocabulary for sampling;
+ *    options sorted_index and return_value).
+ *
+ *  - The lightning-indexer score followed by top-k (NKI pull request "Add
+ *    DeepSeek-V4 CSA attention kernels", "How the algorithm works", steps
+ *    table rows 2 and 3): for every query row t and key position s,
+ *        score[t,s] = sum_h w[t,h] * max(0, q[t,h,:] . k[s,:])
+ *    over a 128-channel bfloat16 key cache shared by all rows, then the k
+ *    highest-scoring positions of each row.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor arguments are DEVICE pointers to caller-owned memory, row-major
+ *    and contiguous.  Nothing is copied to or from the host.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Every call only enqueues work on that stream and returns; no
+ *    call synchronises the host, except ds_get_device_status.
+ *  - The return value is DS_OK (0) or a negative DS_ERR_* code.  Argument
+ *    errors are detected on the host before anything is enqueued.  Errors
+ *    found on the device (a bounded wait that ran out) are recorded in a
+ *    per-device status word that ds_get_device_status reads and clears.
+ *  - Index outputs are int32.  Ties between equal scores go to the lower
+ *    position; -0.0 equals +0.0; every NaN ranks above +inf and all NaNs are
+ *    equal.  Positions s >= valid_len[row] are never selected.  When a row
+ *    has fewer than k eligible positions, the missing slots hold index -1 and
+ *    value / score -inf.
+ *  - The library owns only scratch memory: ds_indexer_topk allocates a
+ *    per-device, grow-only buffer with cudaMalloc on first use (so make the
+ *    first call outside CUDA-graph capture); ds_release frees it.
+ *  - Calls on different streams may run concurrently, except that calls of
+ *    ds_indexer_topk on one device share the scratch buffer and must be
+ *    ordered on one stream.
+ */
+#ifndef DS_TOPK_H
+#define DS_TOPK_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* element types of score rows */
+typedef enum { DS_F32 = 0, DS_BF16 = 1 } ds_dtype;
+
+/* status codes */
+#define DS_OK 0
+#define DS_ERR_ARG (-1)         /* bad argument: null pointer, size, dtype, k, alignment */
+#define DS_ERR_CUDA (-2)        /* a CUDA runtime call or kernel launch failed */
+#define DS_ERR_TIMEOUT (-3)     /* a bounded wait inside a kernel ran out (device status) */
+#define DS_ERR_UNSUPPORTED (-4) /* the current device is not an sm_100 GPU */
+#define DS_ERR_NOMEM (-5)       /* the scratch buffer could not be allocated */
+
+/* limits */
+#define DS_MAX_K 2048            /* largest k of either operation */
+#define DS_INDEXER_DIM 128       /* indexer channels d (fixed) */
+#define DS_INDEXER_MAX_HEADS 64  /* largest number of indexer heads */
+
+/*
+ * ds_topk -- top-k of every row of a [batch, n] score matrix.
+ *   (DeepSelect hub page: the top-k operator of the lightning indexer and of
+ *    sampling; options sorted_index and return_value.)
+ *
+ * scores       device, [batch, n] of `dtype` (float32 or bfloat16), read only.
+ * batch, n     rows and row length; batch >= 1, n >= 1, and one row must fit
+ *              the on-chip budget: n * sizeof(dtype) <= 1.5 MiB
+ *              (n <= 393216 float32 or 786432 bfloat16).
+ * k            1 <= k <= DS_MAX_K.  k may exceed n (extra slots are padding).
+ * dtype        DS_F32 or DS_BF16.
+ * valid_len    device int32 [batch] or NULL.  Row t considers positions
+ *              0 .. min(max(valid_len[t], 0), n) - 1 only.  NULL means n.
+ * out_idx      device int32 [batch, k]: the selected positions.  Without
+ *              sorted_index their order is unspecified; with it they are in
+ *              ascending position order.  Slots past the number of eligible
+ *              positions hold -1.
+ * out_val      device [batch, k] of `dtype`: the stored bit pattern of each
+ *              selected score, -inf in padding slots.  Written only when
+ *              return_value != 0; may be NULL otherwise.
+ * return_value 0 or 1.
+ * sorted_index 0 or 1.
+ * stream       cudaStream_t as void*.
+ * Returns DS_OK, DS_ERR_ARG, DS_ERR_UNSUPPORTED or DS_ERR_CUDA.  Output and
+ * input buffers must not overlap.
+ */
+int ds_topk(const void* scores, int batch, int n, int k, int dtype,
+            const int32_t* valid_len, int32_t* out_idx, void* out_val,
+            int return_value, int sorted_index, void* stream);
+
+/*
+ * ds_indexer_score -- the lightning-indexer score rows, written in full.
+ *   (NKI pull request "Add DeepSeek-V4 CSA attention kernels", "How the
+ *    algorithm works", steps table row 2.)
+ *
+ * q          device bfloat16 [batch, heads, d]: indexer queries.
+ * kcache     device bfloat16 [S, d]: the indexer key cache shared by all rows;
+ *            16-byte aligned.
+ * w          device float32 [batch, heads]: per-row, per-head weights.
+ * batch      >= 1;  heads 1..DS_INDEXER_MAX_HEADS;  d == DS_INDEXER_DIM;  S >= 1.
+ * valid_len  device int32 [batch] or NULL (= S): row t is scored at positions
+ *            s < min(max(valid_len[t], 0), S) only.
+ * out_score  device float32 [batch, S]: score[t, s] for s < valid_len[t];
+ *            positions at or beyond valid_len[t] are set to -inf.
+ * The products are bfloat16 x bfloat16 accumulated in float32 on the tensor
+ * cores; ReLU, weighting and the head sum are float32.
+ * Returns DS_OK, DS_ERR_ARG, DS_ERR_UNSUPPORTED or DS_ERR_CUDA.
+ */
+int ds_indexer_score(const void* q, const void* kcache, const float* w,
+                     int batch, int heads, int d, int S,
+                     const int32_t* valid_len, float* out_score, void* stream);
+
+/*
+ * ds_indexer_topk -- indexer score followed by the top-k positions of each row.
+ *   (NKI pull request "Add DeepSeek-V4 CSA attention kernels", steps table
+ *    rows 2 and 3, and "The top-k on the GPSIMD engine": scoring fused with
+ *    the selection so that the score row does not go back in full.)
+ *
+ * q, kcache, w, batch, heads, d, S, valid_len  as for ds_indexer_score.
+ * k          1 <= k <= DS_MAX_K.
+ * out_idx    device int32 [batch, k]: selected positions, order unspecified,
+ *            -1 in padding slots.
+ * out_score  device float32 [batch, k] or NULL: the float32 score of each
+ *            selected position, -inf in padding slots.
+ * Uses the library's scratch buffer (see above).
+ * Returns DS_OK, DS_ERR_ARG, DS_ERR_UNSUPPORTED, DS_ERR_NOMEM or DS_ERR_CUDA.
+ */
+int ds_indexer_topk(const void* q, const void* kcache, const float* w,
+                    int batch, int heads, int d, int S,
+                    const int32_t* valid_len, int k,
+                    int32_t* out_idx, float* out_score, void* stream);
+
+/*
+ * ds_get_device_status -- synchronise `stream`, then return and clear the
+ * current device's status word: DS_OK, or DS_ERR_TIMEOUT if a kernel's bounded
+ * wait ran out since the last call (its outputs are then unspecified), or
+ * DS_ERR_CUDA if the synchronisation itself failed.
+ * (No counterpart on the pages: the library's error reporting.)
+ */
+int ds_get_device_status(void* stream);
+
+/* ds_strerror -- a static, human-readable name for a status code. */
+const char* ds_strerror(int code);
+
+/* ds_release -- free the scratch buffers of every device this process used.
+ * No call may be in flight. */
+void ds_release(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DS_TOPK_H */

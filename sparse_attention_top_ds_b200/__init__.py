@@ -1,1 +1,17 @@
-"""B200-native selection step of DeepSeek-style sparse attention (placeholder)."""
+"""B200-native selection step of DeepSeek-style sparse attention.
+
+The work happens in libdstopk.so (CUDA kernels for sm_100a behind the C ABI in
+include/ds_topk.h); this package is its Python binding plus seeded input
+generators:
+
+    ds_topk            top-k of bfloat16 / float32 score rows
+    ds_indexer_score   lightning-indexer score rows (tcgen05 tensor cores)
+    ds_indexer_topk    indexer score + top-k
+"""
+
+from ._native import (  # noqa: F401
+    DS_F32, DS_BF16, DS_OK, DS_ERR_ARG, DS_ERR_CUDA, DS_ERR_TIMEOUT, DS_ERR_UNSUPPORTED,
+    DS_ERR_NOMEM, DS_MAX_K, DS_INDEXER_DIM, DS_INDEXER_MAX_HEADS, DsError,
+    ds_topk, ds_indexer_score, ds_indexer_topk, ds_get_device_status, ds_release,
+    strerror, load, lib_path,
+)

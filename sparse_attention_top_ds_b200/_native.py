@@ -1,0 +1,207 @@
+"""ctypes binding of libdstopk.so: argument marshalling only.
+
+Every step of the selection runs in the library's CUDA kernels.  If the shared
+library is missing or cannot be loaded, every call raises; there is no
+fallback implementation.
+"""
+
+import ctypes
+import os
+
+_LIB_PATH = os.environ.get(
+    "DS_TOPK_LIB", os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdstopk.so"))
+
+DS_F32 = 0
+DS_BF16 = 1
+
+DS_OK = 0
+DS_ERR_ARG = -1
+DS_ERR_CUDA = -2
+DS_ERR_TIMEOUT = -3
+DS_ERR_UNSUPPORTED = -4
+DS_ERR_NOMEM = -5
+
+DS_MAX_K = 2048
+DS_INDEXER_DIM = 128
+DS_INDEXER_MAX_HEADS = 64
+
+_lib = None
+
+
+class DsError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        super().__init__(f"{where}: {strerror(code) if _lib is not None else code}")
+
+
+def lib_path():
+    return _LIB_PATH
+
+
+def load():
+    """Load the shared library once; raise if it is not there."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(
+            f"libdstopk.so not found at {_LIB_PATH}; build it with "
+            "`python -m sparse_attention_top_ds_b200.build` (there is no CPU fallback)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i32, i32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
+    lib.ds_topk.argtypes = [vp, i32, i32, i32, i32, i32p, vp, vp, i32, i32, vp]
+    lib.ds_topk.restype = i32
+    lib.ds_indexer_score.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32p, vp, vp]
+    lib.ds_indexer_score.restype = i32
+    lib.ds_indexer_topk.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32p, i32, vp, vp, vp]
+    lib.ds_indexer_topk.restype = i32
+    lib.ds_get_device_status.argtypes = [vp]
+    lib.ds_get_device_status.restype = i32
+    lib.ds_strerror.argtypes = [i32]
+    lib.ds_strerror.restype = ctypes.c_char_p
+    lib.ds_release.argtypes = []
+    lib.ds_release.restype = None
+    _lib = lib
+    return lib
+
+
+def strerror(code):
+    return load().ds_strerror(int(code)).decode()
+
+
+def _check(code, where):
+    if code != DS_OK:
+        raise DsError(code, where)
+
+
+# ------------------------------------------------------------------ raw pointer calls (C ABI)
+
+def ds_topk_raw(scores, batch, n, k, dtype, valid_len, out_idx, out_val, return_value, sorted_index, stream):
+    return load().ds_topk(scores, batch, n, k, dtype, valid_len, out_idx, out_val,
+                          int(return_value), int(sorted_index), stream)
+
+
+def ds_indexer_score_raw(q, kcache, w, batch, heads, d, S, valid_len, out_score, stream):
+    return load().ds_indexer_score(q, kcache, w, batch, heads, d, S, valid_len, out_score, stream)
+
+
+def ds_indexer_topk_raw(q, kcache, w, batch, heads, d, S, valid_len, k, out_idx, out_score, stream):
+    return load().ds_indexer_topk(q, kcache, w, batch, heads, d, S, valid_len, k, out_idx, out_score, stream)
+
+
+def ds_get_device_status(stream=None):
+    return load().ds_get_device_status(_stream_ptr(stream))
+
+
+def ds_release():
+    load().ds_release()
+
+
+# ------------------------------------------------------------------ torch-tensor front end
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _require(t, dtype, name, device=None):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def ds_topk(scores, k, valid_len=None, return_value=True, sorted_index=False,
+            out_idx=None, out_val=None, stream=None):
+    """Top-k of every row of a [batch, n] float32 / bfloat16 CUDA tensor.
+
+    Returns (idx int32 [batch, k], val [batch, k] or None).  Without
+    ``sorted_index`` the order of a row's selection is unspecified.
+    """
+    import torch
+    if scores.dtype == torch.float32:
+        dt = DS_F32
+    elif scores.dtype == torch.bfloat16:
+        dt = DS_BF16
+    else:
+        raise TypeError("scores must be float32 or bfloat16")
+    _require(scores, None, "scores")
+    if scores.dim() != 2:
+        raise ValueError("scores must be [batch, n]")
+    batch, n = scores.shape
+    dev = scores.device
+    if valid_len is not None:
+        _require(valid_len, torch.int32, "valid_len", dev)
+    if out_idx is None:
+        out_idx = torch.empty((batch, k), dtype=torch.int32, device=dev)
+    _require(out_idx, torch.int32, "out_idx", dev)
+    if return_value and out_val is None:
+        out_val = torch.empty((batch, k), dtype=scores.dtype, device=dev)
+    with torch.cuda.device(dev):
+        rc = ds_topk_raw(_ptr(scores), batch, n, k, dt, _ptr(valid_len), _ptr(out_idx),
+                         _ptr(out_val) if return_value else None, return_value, sorted_index,
+                         _stream_ptr(stream))
+    _check(rc, "ds_topk")
+    return out_idx, (out_val if return_value else None)
+
+
+def _indexer_args(q, kcache, w, valid_len):
+    import torch
+    _require(q, torch.bfloat16, "q")
+    dev = q.device
+    _require(kcache, torch.bfloat16, "kcache", dev)
+    _require(w, torch.float32, "w", dev)
+    if q.dim() != 3 or kcache.dim() != 2 or w.dim() != 2:
+        raise ValueError("q [batch,heads,d], kcache [S,d], w [batch,heads]")
+    batch, heads, d = q.shape
+    S = kcache.shape[0]
+    if kcache.shape[1] != d or tuple(w.shape) != (batch, heads):
+        raise ValueError("shape mismatch between q, kcache and w")
+    if valid_len is not None:
+        _require(valid_len, torch.int32, "valid_len", dev)
+    return dev, batch, heads, d, S
+
+
+def ds_indexer_score(q, kcache, w, valid_len=None, out=None, stream=None):
+    """Indexer score rows [batch, S] float32 (-inf at positions >= valid_len)."""
+    import torch
+    dev, batch, heads, d, S = _indexer_args(q, kcache, w, valid_len)
+    if out is None:
+        out = torch.empty((batch, S), dtype=torch.float32, device=dev)
+    _require(out, torch.float32, "out", dev)
+    with torch.cuda.device(dev):
+        rc = ds_indexer_score_raw(_ptr(q), _ptr(kcache), _ptr(w), batch, heads, d, S,
+                                  _ptr(valid_len), _ptr(out), _stream_ptr(stream))
+    _check(rc, "ds_indexer_score")
+    return out
+
+
+def ds_indexer_topk(q, kcache, w, k, valid_len=None, return_score=False,
+                    out_idx=None, out_score=None, stream=None):
+    """Top-k positions of every indexer score row: (idx int32 [batch,k], score f32 [batch,k] or None)."""
+    import torch
+    dev, batch, heads, d, S = _indexer_args(q, kcache, w, valid_len)
+    if out_idx is None:
+        out_idx = torch.empty((batch, k), dtype=torch.int32, device=dev)
+    _require(out_idx, torch.int32, "out_idx", dev)
+    if return_score and out_score is None:
+        out_score = torch.empty((batch, k), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        rc = ds_indexer_topk_raw(_ptr(q), _ptr(kcache), _ptr(w), batch, heads, d, S,
+                                 _ptr(valid_len), k, _ptr(out_idx),
+                                 _ptr(out_score) if return_score else None, _stream_ptr(stream))
+    _check(rc, "ds_indexer_topk")
+    return out_idx, (out_score if return_score else None)

@@ -1,0 +1,243 @@
+// indexer_kernel.cuh -- the lightning-indexer score on the tcgen05 tensor cores.
+//
+// What it computes (NKI pull request "Add DeepSeek-V4 CSA attention kernels",
+// "How the algorithm works", steps table row 2):
+//     score[t, s] = sum_h w[t, h] * max(0, q[t, h, :] . k[s, :]),   d = 128,
+// for s < valid_len[t]; -inf at the other positions.
+//
+// How (B200 design):
+//  * A CTA owns a group of NT query rows and a run of 128-position tiles of
+//    the key cache.  The contraction D[s, (t,h)] = K[s, :] . Q[(t,h), :] is a
+//    dense GEMM with M = 128 positions, N = NT x HP (rows x padded heads),
+//    K = 128 channels: the key tile is operand A, the group's queries are
+//    operand B, both bf16 and K-major in 128-byte-swizzled shared memory
+//    written by TMA; the float32 accumulator lives in TMEM.
+//  * Warp roles: warp 0 issues TMA loads (queries once, key tiles through a
+//    ring of STAGES buffers), warp 1 owns TMEM and issues the MMAs from one
+//    thread, warps 2..9 are the epilogue.  With N <= 256 the accumulator is
+//    double-buffered in TMEM so the epilogue of one tile overlaps the MMAs of
+//    the next.
+//  * Epilogue: after tcgen05.ld each thread holds one position's per-head
+//    products for its rows, so ReLU, the per-head weight (broadcast from
+//    shared memory) and the head sum are a register loop with no shuffles.
+//  * Positions at or past the group's largest valid_len are neither loaded
+//    nor multiplied.
+#pragma once
+
+#include <cuda.h>
+
+#include "ptx.cuh"
+#include "tcgen05.cuh"
+
+namespace dstopk {
+
+struct ScoreParams {
+  const float* w;           // [B, H]
+  const int32_t* valid_len; // [B] or null
+  float* out;               // [B, S]
+  int* status;
+  int B, H, S;
+  int tiles_per_cta;        // 128-position tiles per CTA
+  int ctas_per_group;       // CTAs sharing one group of NT rows
+};
+
+template <int NT, int HP, int STAGES>
+struct ScoreCfg {
+  static constexpr int kN = NT * HP;                 // accumulator columns per tile
+  static constexpr int kNmma = kN < 256 ? kN : 256;  // N of one MMA instruction
+  static constexpr int kNumMma = kN / kNmma;
+  static constexpr int kNbuf = kN <= 256 ? 2 : 1;    // TMEM accumulator buffers
+  static constexpr int kCols = kN * kNbuf;
+  static constexpr int kTmemCols = kCols <= 32 ? 32 : (kCols <= 64 ? 64 : (kCols <= 128 ? 128 : (kCols <= 256 ? 256 : 512)));
+  static constexpr int kQHalf = kN * 128;            // bytes: kN rows x 64 channels x 2 B
+  static constexpr int kKHalf = 128 * 128;           // bytes: 128 positions x 64 channels x 2 B
+  static constexpr int kStage = 2 * kKHalf;
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kThreads = (2 + kEpiWarps) * 32;
+  // shared-memory layout (offsets from a 1024-byte aligned base)
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + 2 * kQHalf;
+  static constexpr int kOffW = kOffK + STAGES * kStage;
+  static constexpr int kOffBar = kOffW + NT * HP * 4;
+  // barriers: qfull, kfull[STAGES], kempty[STAGES], afull[2], aempty[2], tmem slot
+  static constexpr int kBarQ = 0;
+  static constexpr int kBarKFull = 1;
+  static constexpr int kBarKEmpty = 1 + STAGES;
+  static constexpr int kBarAFull = 1 + 2 * STAGES;
+  static constexpr int kBarAEmpty = 3 + 2 * STAGES;
+  static constexpr int kNumBars = 5 + 2 * STAGES;
+  static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffTmemSlot + 16 + 1024;  // + alignment slack
+  static_assert(kN % 16 == 0 && kN <= 512 && kN % kNmma == 0, "bad tile");
+  static_assert(HP % 16 == 0 && HP <= 64, "bad head padding");
+};
+
+template <int NT, int HP, int STAGES>
+__global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
+    indexer_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const ScoreParams p) {
+  using C = ScoreCfg<NT, HP, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  float* w_s = reinterpret_cast<float*>(smem + C::kOffW);
+  const uint32_t bar = sbase + C::kOffBar;
+  auto BAR = [&](int i) -> uint32_t { return bar + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmemSlot);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int group = blockIdx.x / p.ctas_per_group;
+  const int part = blockIdx.x % p.ctas_per_group;
+  const int t0 = group * NT;
+  const int ntiles = (p.S + 127) / 128;
+  const int tile_lo = part * p.tiles_per_cta;
+  const int tile_hi = min(ntiles, tile_lo + p.tiles_per_cta);
+
+  // largest valid length in the group: tiles at or past it are not computed
+  int maxvl = 0;
+  for (int t = 0; t < NT; ++t) {
+    if (t0 + t < p.B) {
+      int v = p.valid_len ? p.valid_len[t0 + t] : p.S;
+      v = v < 0 ? 0 : (v > p.S ? p.S : v);
+      maxvl = max(maxvl, v);
+    }
+  }
+  const int act_hi = min(tile_hi, (maxvl + 127) / 128);
+  const int nact = max(0, act_hi - tile_lo);  // tiles that need the tensor cores
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(C::kBarQ), 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(BAR(C::kBarKFull + s), 1);
+      mbar_init(BAR(C::kBarKEmpty + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(BAR(C::kBarAFull + b), 1);
+      mbar_init(BAR(C::kBarAEmpty + b), C::kEpiWarps);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  // per-head weights of the group (zero for padded heads and absent rows)
+  for (int i = threadIdx.x; i < NT * HP; i += C::kThreads) {
+    const int t = i / HP, h = i % HP;
+    w_s[i] = (t0 + t < p.B && h < p.H) ? p.w[(size_t)(t0 + t) * p.H + h] : 0.0f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0 && nact > 0) {
+      mbar_arrive_expect_tx(BAR(C::kBarQ), 2 * C::kQHalf);
+      tma_load_3d(sbase + C::kOffQ, &tm_q, 0, 0, t0, BAR(C::kBarQ));
+      tma_load_3d(sbase + C::kOffQ + C::kQHalf, &tm_q, 64, 0, t0, BAR(C::kBarQ));
+      for (int i = 0; i < nact; ++i) {
+        const int s = i % STAGES, r = i / STAGES;
+        if (!mbar_wait_bounded(BAR(C::kBarKEmpty + s), (r & 1) ^ 1, p.status)) break;
+        const int pos0 = (tile_lo + i) * 128;
+        mbar_arrive_expect_tx(BAR(C::kBarKFull + s), C::kStage);
+        tma_load_2d(sbase + C::kOffK + s * C::kStage, &tm_k, 0, pos0, BAR(C::kBarKFull + s));
+        tma_load_2d(sbase + C::kOffK + s * C::kStage + C::kKHalf, &tm_k, 64, pos0, BAR(C::kBarKFull + s));
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0 && nact > 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, C::kNmma);
+      bool ok = mbar_wait_bounded(BAR(C::kBarQ), 0, p.status);
+      for (int i = 0; i < nact && ok; ++i) {
+        const int s = i % STAGES, r = i / STAGES;
+        const int b = i % C::kNbuf, u = i / C::kNbuf;
+        if (!mbar_wait_bounded(BAR(C::kBarAEmpty + b), (u & 1) ^ 1, p.status)) break;
+        if (!mbar_wait_bounded(BAR(C::kBarKFull + s), r & 1, p.status)) break;
+        tc_fence_after();
+        const uint32_t a_base = sbase + C::kOffK + s * C::kStage;
+        const uint32_t d_base = tmem_base + (uint32_t)(b * C::kN);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (uint32_t)(kk & 3) * 32u;  // 16 channels = 32 bytes inside the swizzled row
+          const uint32_t a_addr = a_base + (uint32_t)(kk >> 2) * C::kKHalf + koff;
+          const uint64_t adesc = sw128_kmajor_desc(a_addr);
+#pragma unroll
+          for (int j = 0; j < C::kNumMma; ++j) {
+            const uint32_t b_addr = sbase + C::kOffQ + (uint32_t)(kk >> 2) * C::kQHalf +
+                                    (uint32_t)(j * C::kNmma) * 128u + koff;
+            mma_bf16_ss(d_base + (uint32_t)(j * C::kNmma), adesc, sw128_kmajor_desc(b_addr), idesc,
+                        kk > 0 ? 1u : 0u);
+          }
+        }
+        mma_commit(BAR(C::kBarKEmpty + s));
+        mma_commit(BAR(C::kBarAFull + b));
+      }
+    }
+  } else {
+    // ---------------- epilogue: 8 warps; TMEM lane quarter = warp % 4
+    const int e = warp - 2;
+    const int qd = warp & 3;
+    const int hf = e >> 2;  // which half of the group's rows
+    const int row = qd * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
+    constexpr int TPH = (NT + 1) / 2;  // rows per epilogue half
+    int vl[TPH];
+#pragma unroll
+    for (int j = 0; j < TPH; ++j) {
+      const int tl = hf * TPH + j;
+      const int t = t0 + tl;
+      int v = 0;
+      if (tl < NT && t < p.B) {
+        v = p.valid_len ? p.valid_len[t] : p.S;
+        v = v < 0 ? 0 : (v > p.S ? p.S : v);
+      }
+      vl[j] = v;
+    }
+    for (int i = 0; i < nact; ++i) {
+      const int b = i % C::kNbuf, u = i / C::kNbuf;
+      if (!mbar_wait_bounded(BAR(C::kBarAFull + b), u & 1, p.status)) break;  // status records the timeout
+      tc_fence_after();
+      const int s = (tile_lo + i) * 128 + row;
+#pragma unroll
+      for (int j = 0; j < TPH; ++j) {
+        const int tl = hf * TPH + j;  // row inside the group
+        if (tl >= NT) break;
+        const uint32_t col = tmem_base + lane_addr + (uint32_t)(b * C::kN + tl * HP);
+        uint32_t r[HP];
+#pragma unroll
+        for (int c = 0; c < HP; c += 16) tmem_ld16(col + (uint32_t)c, *reinterpret_cast<uint32_t(*)[16]>(r + c));
+        tmem_wait_ld();
+        float acc = 0.0f;
+#pragma unroll
+        for (int x = 0; x < HP; ++x) acc = fmaf(w_s[tl * HP + x], fmaxf(__uint_as_float(r[x]), 0.0f), acc);
+        const int t = t0 + tl;
+        if (t < p.B && s < p.S) p.out[(size_t)t * p.S + s] = (s < vl[j]) ? acc : -INFINITY;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::kBarAEmpty + b));
+    }
+    // tiles past the group's valid lengths: no products, -inf
+    for (int tile = act_hi > tile_lo ? act_hi : tile_lo; tile < tile_hi; ++tile) {
+      const int s = tile * 128 + row;
+#pragma unroll
+      for (int j = 0; j < TPH; ++j) {
+        const int tl = hf * TPH + j;
+        const int t = t0 + tl;
+        if (tl < NT && t < p.B && s < p.S) p.out[(size_t)t * p.S + s] = -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+}  // namespace dstopk

@@ -1,0 +1,352 @@
+// lib.cu -- the C ABI of libdstopk.so (declared in include/ds_topk.h):
+// argument checks, launch-shape choice and kernel launches.  One translation
+// unit holds every kernel, so device symbols (the status word) resolve here.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "../../include/ds_topk.h"
+#include "ptx.cuh"
+#include "topk_kernel.cuh"
+#include "indexer_kernel.cuh"
+
+namespace dstopk {
+
+// Per-device status word: kernels record the first device-side error here.
+static __device__ int g_status;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  bool supported = false;
+  int num_sms = 0;
+  int* status = nullptr;     // device address of g_status on this device
+  void* scratch = nullptr;   // grow-only scratch for ds_indexer_topk
+  size_t scratch_bytes = 0;
+};
+
+static std::mutex g_mu;
+static DeviceState g_dev[kMaxDevices];
+
+static cudaError_t indexer_setup();
+
+// Set-up once per device, with that device current: capability check, the
+// status word's address, and the kernels' shared-memory limits.
+static int device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DS_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (!s.ready) {
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return DS_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DS_ERR_CUDA;
+    s.supported = (major == 10);
+    s.num_sms = sms;
+    if (s.supported) {
+      if (cudaGetSymbolAddress(reinterpret_cast<void**>(&s.status), g_status) != cudaSuccess) return DS_ERR_CUDA;
+      const int smem_max = 227 * 1024;
+      cudaError_t e = cudaSuccess;
+      e = cudaFuncSetAttribute(topk_cluster_kernel<F32Keys, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(topk_cluster_kernel<F32Keys, 512>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(topk_cluster_kernel<BF16Keys, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(topk_cluster_kernel<BF16Keys, 512>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
+      if (e == cudaSuccess) e = indexer_setup();
+      if (e != cudaSuccess) return DS_ERR_CUDA;
+    }
+    s.ready = true;
+  }
+  if (!s.supported) return DS_ERR_UNSUPPORTED;
+  *out = &s;
+  return DS_OK;
+}
+
+// ------------------------------------------------------------------ top-k
+
+struct TopkShape {
+  int cluster;   // CTAs per row
+  int slice;     // elements per CTA
+  int threads;   // threads per CTA
+};
+
+// Launch shape: split a row over a cluster until a slice is small enough to
+// sit in shared memory next to other CTAs, and until the grid fills the GPU
+// (about two CTAs per SM), but never below 4 KiB per slice.
+static bool choose_topk_shape(int batch, int n, int elem, int num_sms, TopkShape* out) {
+  int C = 1;
+  const long target = 2L * num_sms;
+  const char* force = getenv("DS_TOPK_CLUSTER");  // tuning sweeps only
+  if (force) {
+    C = atoi(force);
+    if (C != 1 && C != 2 && C != 4 && C != 8) C = 8;
+  } else {
+    while (C < 8) {
+      const long sb = (long)((n + C - 1) / C) * elem;
+      const bool too_big = sb > 48 * 1024;
+      const bool too_few = (long)batch * C < target && sb > 4096;
+      if (!too_big && !too_few) break;
+      C *= 2;
+    }
+  }
+  int slice = (n + C - 1) / C;
+  slice = (slice + 7) / 8 * 8;
+  if ((long)slice * elem > kMaxSliceBytes) return false;
+  out->cluster = C;
+  out->slice = slice;
+  out->threads = ((long)slice * elem >= 32 * 1024) ? 512 : 256;
+  return true;
+}
+
+template <class K, int NT>
+static cudaError_t launch_topk(const TopkParams& p, int C, cudaStream_t st) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)(p.batch * C), 1, 1);
+  cfg.blockDim = dim3(NT, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)topk_smem_bytes(p.slice * K::kBytes);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, topk_cluster_kernel<K, NT>, p);
+}
+
+static int topk_enqueue(const void* scores, int batch, int n, int k, int dtype, const int32_t* valid_len,
+                        int32_t* out_idx, void* out_val, int return_value, cudaStream_t st, DeviceState* s) {
+  const int elem = dtype == DS_F32 ? 4 : 2;
+  TopkShape sh;
+  if (!choose_topk_shape(batch, n, elem, s->num_sms, &sh)) return DS_ERR_ARG;
+  TopkParams p;
+  p.scores = scores;
+  p.valid_len = valid_len;
+  p.out_idx = out_idx;
+  p.out_val = out_val;
+  p.status = s->status;
+  p.batch = batch;
+  p.n = n;
+  p.k = k;
+  p.slice = sh.slice;
+  p.return_value = return_value ? 1 : 0;
+  cudaError_t e;
+  if (dtype == DS_F32)
+    e = sh.threads == 512 ? launch_topk<F32Keys, 512>(p, sh.cluster, st) : launch_topk<F32Keys, 256>(p, sh.cluster, st);
+  else
+    e = sh.threads == 512 ? launch_topk<BF16Keys, 512>(p, sh.cluster, st)
+                          : launch_topk<BF16Keys, 256>(p, sh.cluster, st);
+  return e == cudaSuccess ? DS_OK : DS_ERR_CUDA;
+}
+
+
+// ------------------------------------------------------------------ indexer
+
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+template <int NT, int HP, int ST>
+static cudaError_t set_score_smem() {
+  return cudaFuncSetAttribute(indexer_score_kernel<NT, HP, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              ScoreCfg<NT, HP, ST>::kSmemBytes);
+}
+
+// Called once per device from device_state (under its lock).
+static cudaError_t indexer_setup() {
+  if (!g_encode) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  cudaError_t e = set_score_smem<1, 64, 4>();
+  if (e == cudaSuccess) e = set_score_smem<2, 64, 4>();
+  if (e == cudaSuccess) e = set_score_smem<4, 64, 4>();
+  if (e == cudaSuccess) e = set_score_smem<8, 64, 2>();
+  if (e == cudaSuccess) e = set_score_smem<8, 32, 4>();
+  if (e == cudaSuccess) e = set_score_smem<8, 16, 4>();
+  return e;
+}
+
+// bf16 tensor maps with 128-byte swizzle: queries [B][H][128] in boxes of
+// (64 channels, HP heads, NT rows); keys [S][128] in boxes of (64, 128).
+static bool encode_maps(const void* q, const void* kc, int B, int H, int S, int HP, int NT, CUtensorMap* tq,
+                        CUtensorMap* tk) {
+  cuuint64_t qdims[3] = {128, (cuuint64_t)H, (cuuint64_t)B};
+  cuuint64_t qstr[2] = {256, (cuuint64_t)H * 256};
+  cuuint32_t qbox[3] = {64, (cuuint32_t)HP, (cuuint32_t)NT};
+  cuuint32_t one3[3] = {1, 1, 1};
+  CUresult r = g_encode(tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), qdims, qstr, qbox, one3,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  cuuint64_t kdims[2] = {128, (cuuint64_t)S};
+  cuuint64_t kstr[1] = {256};
+  cuuint32_t kbox[2] = {64, 128};
+  cuuint32_t one2[2] = {1, 1};
+  r = g_encode(tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kc), kdims, kstr, kbox, one2,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int NT, int HP, int ST>
+static int launch_score(const void* q, const void* kc, const float* w, int B, int H, int S, const int32_t* vl,
+                        float* out, cudaStream_t st, DeviceState* s) {
+  using Cfg = ScoreCfg<NT, HP, ST>;
+  CUtensorMap tq, tk;
+  if (!encode_maps(q, kc, B, H, S, HP, NT, &tq, &tk)) return DS_ERR_ARG;
+  const int ntiles = (S + 127) / 128;
+  const int groups = (B + NT - 1) / NT;
+  // spread one group's tiles over several CTAs only while there are fewer
+  // groups than SMs
+  long tpc = ((long)groups * ntiles + s->num_sms - 1) / s->num_sms;
+  if (tpc < 1) tpc = 1;
+  if (tpc > ntiles) tpc = ntiles;
+  const int cpg = (int)((ntiles + tpc - 1) / tpc);
+  ScoreParams p;
+  p.w = w;
+  p.valid_len = vl;
+  p.out = out;
+  p.status = s->status;
+  p.B = B;
+  p.H = H;
+  p.S = S;
+  p.tiles_per_cta = (int)tpc;
+  p.ctas_per_group = cpg;
+  indexer_score_kernel<NT, HP, ST><<<groups * cpg, Cfg::kThreads, Cfg::kSmemBytes, st>>>(tq, tk, p);
+  return cudaGetLastError() == cudaSuccess ? DS_OK : DS_ERR_CUDA;
+}
+
+static int score_enqueue(const void* q, const void* kc, const float* w, int B, int H, int S, const int32_t* vl,
+                         float* out, cudaStream_t st, DeviceState* s) {
+  if (H > 32) {
+    if (B == 1) return launch_score<1, 64, 4>(q, kc, w, B, H, S, vl, out, st, s);
+    if (B == 2) return launch_score<2, 64, 4>(q, kc, w, B, H, S, vl, out, st, s);
+    if (B <= 4 || B > 8) return launch_score<4, 64, 4>(q, kc, w, B, H, S, vl, out, st, s);
+    return launch_score<8, 64, 2>(q, kc, w, B, H, S, vl, out, st, s);
+  }
+  if (H > 16) return launch_score<8, 32, 4>(q, kc, w, B, H, S, vl, out, st, s);
+  return launch_score<8, 16, 4>(q, kc, w, B, H, S, vl, out, st, s);
+}
+
+static int indexer_check(const void* q, const void* kc, const float* w, int B, int H, int d, int S) {
+  if (!q || !kc || !w || B <= 0 || H <= 0 || H > DS_INDEXER_MAX_HEADS || d != DS_INDEXER_DIM || S <= 0)
+    return DS_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(q) & 15u) || (reinterpret_cast<uintptr_t>(kc) & 15u) ||
+      (reinterpret_cast<uintptr_t>(w) & 3u))
+    return DS_ERR_ARG;
+  return DS_OK;
+}
+
+// Grow-only per-device scratch; the caller holds no lock.
+static void* get_scratch(DeviceState* s, size_t bytes) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (s->scratch_bytes >= bytes) return s->scratch;
+  if (s->scratch) cudaFree(s->scratch);
+  s->scratch = nullptr;
+  s->scratch_bytes = 0;
+  void* p = nullptr;
+  if (cudaMalloc(&p, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  s->scratch = p;
+  s->scratch_bytes = bytes;
+  return p;
+}
+
+}  // namespace dstopk
+
+using namespace dstopk;
+
+extern "C" int ds_topk(const void* scores, int batch, int n, int k, int dtype, const int32_t* valid_len,
+                       int32_t* out_idx, void* out_val, int return_value, int sorted_index, void* stream) {
+  if (!scores || !out_idx || batch <= 0 || n <= 0 || k <= 0 || k > DS_MAX_K) return DS_ERR_ARG;
+  if (dtype != DS_F32 && dtype != DS_BF16) return DS_ERR_ARG;
+  if (return_value && !out_val) return DS_ERR_ARG;
+  if ((long)n * (dtype == DS_F32 ? 4 : 2) > 8L * kMaxSliceBytes) return DS_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(scores) & (dtype == DS_F32 ? 3u : 1u)) != 0) return DS_ERR_ARG;
+  (void)sorted_index;  // the selection is always written in ascending position order
+  DeviceState* s = nullptr;
+  const int rc = device_state(&s);
+  if (rc != DS_OK) return rc;
+  return topk_enqueue(scores, batch, n, k, dtype, valid_len, out_idx, out_val, return_value,
+                      static_cast<cudaStream_t>(stream), s);
+}
+
+extern "C" int ds_get_device_status(void* stream) {
+  DeviceState* s = nullptr;
+  const int rc = device_state(&s);
+  if (rc != DS_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int host = 0;
+  if (cudaMemcpyAsync(&host, s->status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return DS_ERR_CUDA;
+  if (cudaMemsetAsync(s->status, 0, sizeof(int), st) != cudaSuccess) return DS_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DS_ERR_CUDA;
+  return host;
+}
+
+extern "C" const char* ds_strerror(int code) {
+  switch (code) {
+    case DS_OK: return "DS_OK";
+    case DS_ERR_ARG: return "DS_ERR_ARG: invalid argument";
+    case DS_ERR_CUDA: return "DS_ERR_CUDA: CUDA runtime error";
+    case DS_ERR_TIMEOUT: return "DS_ERR_TIMEOUT: a bounded device wait ran out";
+    case DS_ERR_UNSUPPORTED: return "DS_ERR_UNSUPPORTED: device is not sm_100";
+    case DS_ERR_NOMEM: return "DS_ERR_NOMEM: scratch allocation failed";
+    default: return "unknown status";
+  }
+}
+
+extern "C" void ds_release(void) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) cur = -1;
+  for (int d = 0; d < kMaxDevices; ++d) {
+    if (g_dev[d].scratch) {
+      if (cudaSetDevice(d) == cudaSuccess) cudaFree(g_dev[d].scratch);
+      g_dev[d].scratch = nullptr;
+      g_dev[d].scratch_bytes = 0;
+    }
+  }
+  if (cur >= 0) cudaSetDevice(cur);
+}
+
+extern "C" int ds_indexer_score(const void* q, const void* kcache, const float* w, int batch, int heads, int d,
+                                int S, const int32_t* valid_len, float* out_score, void* stream) {
+  int rc = indexer_check(q, kcache, w, batch, heads, d, S);
+  if (rc != DS_OK) return rc;
+  if (!out_score) return DS_ERR_ARG;
+  DeviceState* s = nullptr;
+  rc = device_state(&s);
+  if (rc != DS_OK) return rc;
+  return score_enqueue(q, kcache, w, batch, heads, S, valid_len, out_score, static_cast<cudaStream_t>(stream), s);
+}
+
+extern "C" int ds_indexer_topk(const void* q, const void* kcache, const float* w, int batch, int heads, int d, int S,
+                               const int32_t* valid_len, int k, int32_t* out_idx, float* out_score, void* stream) {
+  int rc = indexer_check(q, kcache, w, batch, heads, d, S);
+  if (rc != DS_OK) return rc;
+  if (!out_idx || k <= 0 || k > DS_MAX_K) return DS_ERR_ARG;
+  if ((long)S * 4 > 8L * kMaxSliceBytes) return DS_ERR_ARG;
+  DeviceState* s = nullptr;
+  rc = device_state(&s);
+  if (rc != DS_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* scores = static_cast<float*>(get_scratch(s, (size_t)batch * (size_t)S * sizeof(float)));
+  if (!scores) return DS_ERR_NOMEM;
+  rc = score_enqueue(q, kcache, w, batch, heads, S, valid_len, scores, st, s);
+  if (rc != DS_OK) return rc;
+  return topk_enqueue(scores, batch, S, k, DS_F32, valid_len, out_idx, out_score, out_score != nullptr, st, s);
+}

@@ -1,0 +1,85 @@
+"""The C-ABI library builds, loads and exports every entry point that
+include/ds_topk.h declares; host-side argument checks answer without a GPU;
+the Python binding fails loudly when the library is missing (CPU only)."""
+
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ds_topk.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_attention_top_ds_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ds_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_entry_points()
+    for n in ("ds_topk", "ds_indexer_score", "ds_indexer_topk", "ds_get_device_status", "ds_strerror",
+              "ds_release"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_entry_points():
+        assert hasattr(lib, name), f"{name} is declared but not exported"
+
+
+def test_exported_symbols_have_c_linkage(lib):
+    from sparse_attention_top_ds_b200 import build
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (ds_\w+)$", out, flags=re.M))
+    assert set(declared_entry_points()) <= exported
+
+
+def test_strerror(lib):
+    lib.ds_strerror.restype = ctypes.c_char_p
+    assert lib.ds_strerror(0) == b"DS_OK"
+    assert b"argument" in lib.ds_strerror(-1)
+    assert b"unknown" in lib.ds_strerror(12345)
+
+
+def test_argument_errors_need_no_gpu(lib):
+    # every one of these is rejected on the host before any CUDA call
+    vp = ctypes.c_void_p
+    fake = vp(0x100000)
+    lib.ds_topk.restype = ctypes.c_int
+    lib.ds_topk.argtypes = [vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp,
+                            ctypes.c_int, ctypes.c_int, vp]
+    assert lib.ds_topk(None, 1, 10, 5, 0, None, fake, fake, 1, 0, None) == -1      # null scores
+    assert lib.ds_topk(fake, 0, 10, 5, 0, None, fake, fake, 1, 0, None) == -1      # batch
+    assert lib.ds_topk(fake, 1, 10, 0, 0, None, fake, fake, 1, 0, None) == -1      # k = 0
+    assert lib.ds_topk(fake, 1, 10, 2049, 0, None, fake, fake, 1, 0, None) == -1   # k > max
+    assert lib.ds_topk(fake, 1, 10, 5, 7, None, fake, fake, 1, 0, None) == -1      # dtype
+    assert lib.ds_topk(fake, 1, 10, 5, 0, None, fake, None, 1, 0, None) == -1      # out_val missing
+    assert lib.ds_topk(fake, 1, 400000, 5, 0, None, fake, fake, 1, 0, None) == -1  # row too long
+    assert lib.ds_topk(vp(0x100001), 1, 10, 5, 0, None, fake, fake, 1, 0, None) == -1  # misaligned
+    lib.ds_indexer_topk.restype = ctypes.c_int
+    lib.ds_indexer_topk.argtypes = [vp, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp,
+                                    ctypes.c_int, vp, vp, vp]
+    assert lib.ds_indexer_topk(fake, fake, fake, 1, 64, 64, 100, None, 10, fake, None, None) == -1   # d
+    assert lib.ds_indexer_topk(fake, fake, fake, 1, 65, 128, 100, None, 10, fake, None, None) == -1  # heads
+    assert lib.ds_indexer_topk(fake, fake, fake, 1, 64, 128, 100, None, 0, fake, None, None) == -1   # k
+    assert lib.ds_indexer_topk(fake, vp(0x100008), fake, 1, 64, 128, 100, None, 10, fake, None, None) == -1
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    code = ("import sparse_attention_top_ds_b200 as ds\n"
+            "try:\n    ds.load()\nexcept RuntimeError as e:\n    print('RAISED', e)\n")
+    env = dict(os.environ, DS_TOPK_LIB=str(tmp_path / "missing.so"), PYTHONPATH=ROOT)
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, cwd=ROOT)
+    assert "RAISED" in out.stdout and "no CPU fallback" in out.stdout

@@ -1,0 +1,167 @@
+"""GPU parity of ds_indexer_score and ds_indexer_topk (through the C ABI) with
+the float64 oracle.
+
+Bars (products are bf16 x bf16 accumulated in float32):
+  * scores: |gpu - oracle| <= 1e-2 * |oracle| + 1e-6 * rowmax, and the tighter
+    float32 accumulation bound (d + H) * 2^-23 * sum|w * relu(q.k)| ... checked
+    as 1e-4 relative on the row scale;
+  * exact-arithmetic inputs (small integer q, k; power-of-two w): every float32
+    partial sum is exact, so scores match bit for bit and the selected index
+    sets match exactly;
+  * selection on random inputs: min(k, valid_len) distinct in-range indices,
+    each with oracle score >= the oracle's k-th value - 1e-2 * |k-th value|, and
+    returned scores within 1e-2 relative of the oracle's.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_attention_top_ds_b200 as ds
+from sparse_attention_top_ds_b200 import inputs
+from gpu_util import bf16_to_device, f32_to_device, i32_to_device
+
+pytestmark = pytest.mark.gpu
+
+REL_TOL = 1e-2
+
+
+def dev_inputs(q, kc, w, vl):
+    return (bf16_to_device(q), bf16_to_device(kc), f32_to_device(w),
+            None if vl is None else i32_to_device(vl))
+
+
+def check_scores(q, kc, w, vl, strict=True):
+    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
+    got = ds.ds_indexer_score(qd, kd, wd, valid_len=vd).cpu().numpy().astype(np.float64)
+    torch.cuda.synchronize()
+    assert ds.ds_get_device_status() == ds.DS_OK
+    ref = oracle.indexer_scores(q, kc, w, vl)
+    B, S = ref.shape
+    for t in range(B):
+        L = S if vl is None else max(0, min(int(vl[t]), S))
+        assert np.all(np.isneginf(got[t, L:])), f"row {t}: positions past valid_len must be -inf"
+        if L == 0:
+            continue
+        r, g = ref[t, :L], got[t, :L]
+        scale = max(np.abs(r).max(), 1e-30)
+        err = np.abs(g - r)
+        assert np.all(err <= REL_TOL * np.abs(r) + 1e-6 * scale), f"row {t}: max err {err.max()}"
+        if strict:
+            assert err.max() <= 1e-4 * scale, f"row {t}: error {err.max() / scale} of the row scale"
+    return got, ref
+
+
+def check_selection(q, kc, w, vl, k, idx, score):
+    ref = oracle.indexer_scores(q, kc, w, vl)
+    B, S = ref.shape
+    for t in range(B):
+        L = S if vl is None else max(0, min(int(vl[t]), S))
+        m = min(k, L)
+        sel = idx[t]
+        assert int((sel >= 0).sum()) == m and np.all(sel[m:] == -1), f"row {t}: count / padding"
+        s = sel[:m]
+        assert len(np.unique(s)) == m and np.all((s >= 0) & (s < L)), f"row {t}: distinct in-range"
+        if m == 0:
+            continue
+        vk = np.sort(ref[t, :L])[::-1][m - 1]
+        assert np.all(ref[t, s] >= vk - REL_TOL * abs(vk)), f"row {t}: a selected score is below the k-th"
+        if score is not None:
+            rs = ref[t, s]
+            assert np.all(np.abs(score[t, :m] - rs) <= REL_TOL * np.abs(rs) + 1e-6 * max(abs(vk), 1e-30))
+            assert np.all(np.isneginf(score[t, m:]))
+
+
+# ---------------------------------------------------------------- scores
+
+@pytest.mark.parametrize("B,H,S", [(1, 64, 128), (3, 64, 1000), (8, 64, 4096), (9, 64, 777),
+                                   (5, 32, 300), (2, 16, 256), (4, 8, 129), (3, 1, 200), (2, 48, 260)])
+def test_scores_random(cuda_device, B, H, S):
+    q, kc, w = inputs.indexer_factors(seed=100 + B * H + S, batch=B, n=S, heads=H)
+    check_scores(q, kc, w, None)
+
+
+def test_scores_valid_len(cuda_device):
+    q, kc, w = inputs.indexer_factors(seed=5, batch=8, n=3000, heads=64)
+    vl = np.array([0, 1, 127, 128, 129, 2999, 3000, 5000], dtype=np.int32)
+    check_scores(q, kc, w, vl)
+
+
+def exact_inputs(seed, B, H, S):
+    g = np.random.default_rng(seed)
+    q = inputs.f32_to_bf16_bits(g.integers(-4, 5, size=(B, H, 128)).astype(np.float32))
+    kc = inputs.f32_to_bf16_bits(g.integers(-4, 5, size=(S, 128)).astype(np.float32))
+    w = g.choice(np.array([0.25, 0.5, 1.0, 2.0], dtype=np.float32), size=(B, H))
+    return q, kc, w
+
+
+@pytest.mark.parametrize("B,H,S", [(8, 64, 2048), (13, 64, 700), (2, 64, 33), (8, 32, 500)])
+def test_scores_exact_arithmetic(cuda_device, B, H, S):
+    q, kc, w = exact_inputs(B * 7 + S, B, H, S)
+    got, ref = check_scores(q, kc, w, None)
+    assert np.array_equal(got, ref), "exact-arithmetic scores must match bit for bit"
+
+
+# ---------------------------------------------------------------- selection
+
+@pytest.mark.parametrize("B,H,S,k", [(8, 64, 2048, 1024), (13, 64, 700, 100), (8, 32, 500, 499)])
+def test_topk_exact_arithmetic(cuda_device, B, H, S, k):
+    q, kc, w = exact_inputs(B * 11 + S, B, H, S)
+    qd, kd, wd, _ = dev_inputs(q, kc, w, None)
+    idx, score = ds.ds_indexer_topk(qd, kd, wd, k, return_score=True)
+    ref_idx, ref_scores = oracle.indexer_topk(q, kc, w, k)
+    idx = idx.cpu().numpy()
+    score = score.cpu().numpy()
+    for t in range(B):
+        m = int((ref_idx[t] >= 0).sum())
+        assert np.array_equal(np.sort(idx[t, :m]), np.sort(ref_idx[t, :m])), f"row {t}"
+        assert np.array_equal(score[t, :m].astype(np.float64), ref_scores[t, idx[t, :m]])
+
+
+def test_decode_8x64x128_vs_32768_k1024(cuda_device):
+    q, kc, w, vl = inputs.decode()
+    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
+    idx, score = ds.ds_indexer_topk(qd, kd, wd, 1024, valid_len=vd, return_score=True)
+    torch.cuda.synchronize()
+    assert ds.ds_get_device_status() == ds.DS_OK
+    check_selection(q, kc, w, vl, 1024, idx.cpu().numpy(), score.cpu().numpy())
+
+
+def test_prefill_4096_rows_sampled(cuda_device):
+    q, kc, w, vl = inputs.prefill()
+    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
+    idx, score = ds.ds_indexer_topk(qd, kd, wd, 2048, valid_len=vd, return_score=True)
+    torch.cuda.synchronize()
+    assert ds.ds_get_device_status() == ds.DS_OK
+    rows = inputs.sample_rows(inputs.SEED_PREFILL, q.shape[0], 64)
+    check_selection(q[rows], kc, w[rows], vl[rows], 2048, idx.cpu().numpy()[rows], score.cpu().numpy()[rows])
+    # every row: min(k, valid_len) distinct in-range indices
+    allidx = idx.cpu().numpy()
+    assert np.all((allidx >= 0) & (allidx < vl[:, None]))
+    srt = np.sort(allidx, axis=1)
+    assert np.all(np.diff(srt, axis=1) > 0)
+
+
+@pytest.mark.parametrize("B,H,S,k", [(3, 64, 1000, 2048), (9, 64, 5000, 64), (1, 64, 300, 1), (6, 16, 4000, 512)])
+def test_topk_valid_len_and_padding(cuda_device, B, H, S, k):
+    q, kc, w = inputs.indexer_factors(seed=B + S + k, batch=B, n=S, heads=H)
+    g = np.random.default_rng(B)
+    vl = g.integers(-2, S + 10, size=B).astype(np.int32)
+    vl[0] = 0
+    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
+    idx, score = ds.ds_indexer_topk(qd, kd, wd, k, valid_len=vd, return_score=True)
+    check_selection(q, kc, w, vl, k, idx.cpu().numpy(), score.cpu().numpy())
+
+
+def test_indexer_argument_errors(cuda_device):
+    q = torch.zeros((2, 64, 64), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((100, 64), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((2, 64), dtype=torch.float32, device="cuda")
+    with pytest.raises(ds.DsError):
+        ds.ds_indexer_score(q, kc, w)            # d != 128
+    q = torch.zeros((2, 65, 128), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((100, 128), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((2, 65), dtype=torch.float32, device="cuda")
+    with pytest.raises(ds.DsError):
+        ds.ds_indexer_topk(q, kc, w, 10)         # heads > 64
