@@ -1,0 +1,416 @@
+"""Benchmark of the sparse-attention selection step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole selection path over one batch of synthetic,
+seeded input:
+  * top-k of the sampling workload (64 rows x 129280 float32 logits ~ N(0, 9)
+    with 20 planted +15 outliers per row) at k = 1024 and at k = 64, values
+    and indices, unsorted;
+  * the decode indexer + top-k (8 query rows x 64 heads x 128 bf16 against one
+    bf16 key cache of 32768 positions, valid_len ~ U{4096..32768}, k = 1024).
+The headline value is the top-k effective HBM bandwidth (algorithmic bytes /
+device time, GB/s); the decode indexer + top-k time is reported in
+microseconds per decode step beside it.  Inputs rotate through enough copies
+(> 2x the 126 MB L2) that every call reads HBM.  With N > 1 (torchrun, one
+process per GPU) every rank processes its own batch (weak scaling, no data
+collective); the value is the total over ranks divided by the slowest rank's
+time.
+
+``--impl reference`` times the CPU oracle (float64, single thread) on a bounded
+sample of the same workload and prints the same line with "impl": "reference".
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "top-k effective HBM GB/s (% of peak); indexer+top-k µs per decode step"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+L2_BYTES = 126 * 1024 * 1024
+
+SAMPLING = dict(batch=64, n=129280, ks=(1024, 64))
+DECODE = dict(batch=8, heads=64, d=128, S=32768, k=1024)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def topk_bytes(batch, n, k, elem=4):
+    """Algorithmic bytes of one top-k call: read every score once, write k
+    (int32 index + value) per row."""
+    return batch * n * elem + batch * k * (4 + elem)
+
+
+def decode_bytes_flops(vl, heads, d, k):
+    """Algorithmic bytes and FLOPs of one decode indexer + top-k call."""
+    maxvl = int(np.max(vl))
+    B = len(vl)
+    bytes_ = maxvl * d * 2 + B * heads * d * 2 + B * heads * 4 + B * 4 + B * k * 4
+    flops = 2 * heads * d * int(np.sum(vl))
+    return bytes_, flops
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            parts = [x.strip() for x in l.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_uuid(dev):
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+
+def oracle_sample(seconds=10.0, decode_rows=8):
+    """Time the CPU oracle (single thread) on a bounded sample of the workload.
+
+    Top-k: whole rows of the sampling workload at k = 1024 and 64, as many as
+    fit in `seconds`.  Decode: the float64 indexer score + top-k of the decode
+    workload's rows.  Returns a dict with GB/s, rows and microseconds."""
+    from threadpoolctl import threadpool_limits
+    import oracle
+    from sparse_attention_top_ds_b200 import inputs
+    x, _ = inputs.sampling()
+    q, kc, w, vl = inputs.decode()
+    with threadpool_limits(limits=1):
+        done_bytes, rows, t0 = 0, 0, time.perf_counter()
+        while time.perf_counter() - t0 < seconds and rows < 2 * x.shape[0]:
+            t = rows % x.shape[0]
+            k = SAMPLING["ks"][(rows // x.shape[0]) % 2]
+            oracle.topk_rows(x[t:t + 1], "f32", k)
+            done_bytes += topk_bytes(1, x.shape[1], k)
+            rows += 1
+        t_topk = time.perf_counter() - t0
+        t1 = time.perf_counter()
+        oracle.indexer_topk(q[:decode_rows], kc, w[:decode_rows], DECODE["k"], vl[:decode_rows])
+        t_dec = time.perf_counter() - t1
+    return {"topk_gbs": done_bytes / t_topk / 1e9, "topk_rows": rows, "topk_s": t_topk,
+            "decode_us": t_dec * 1e6 * (DECODE["batch"] / decode_rows), "decode_rows": decode_rows}
+
+
+# ------------------------------------------------------------------ distributed helpers
+
+def dist_setup(backend):
+    import torch.distributed as dist
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return (dist.get_rank() if dist.is_initialized() else 0), ws
+
+
+def max_over_ranks(values, device):
+    """Element-wise max of a list of floats over all ranks."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_initialized():
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ arms
+
+def run_reference(args):
+    rank, ws = dist_setup("gloo")
+    if rank != 0:
+        return
+    r = oracle_sample(seconds=max(3.0, min(20.0, 0.2 * args.steps)))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(r["topk_gbs"], 6), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "decode_us_per_step": round(r["decode_us"], 1),
+        "config": {"workload": "sampling top-k 64x129280 f32 k in {1024,64} + decode indexer 8x64x128 vs 32768 "
+                               "k=1024 (bounded oracle sample)"},
+        "cpu_baseline": {"value": round(r["topk_gbs"], 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{r['topk_rows']} sampling rows (k=1024/64) + {r['decode_rows']} decode rows"},
+        "e2e": {"value": round(r["topk_gbs"], 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+    import sparse_attention_top_ds_b200 as ds
+    from sparse_attention_top_ds_b200 import inputs
+
+    rank, ws = dist_setup("nccl")
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    hbm_gbs, tflops, tflops_sus, peak_src = load_peaks()
+
+    # ---- inputs (each rank its own seeded batch), resident in HBM
+    x_host, _ = inputs.sampling(seed=inputs.SEED_SAMPLING + rank)
+    xb = x_host.nbytes
+    R = max(3, -(-2 * L2_BYTES // xb) + 1)
+    xs = [torch.from_numpy(x_host).to(dev) for _ in range(R)]
+    xs2 = [torch.from_numpy(x_host).to(dev) for _ in range(R)]   # the k=64 phase rotates its own copies
+    q, kc, w, vl = inputs.decode(seed=inputs.SEED_DECODE + rank)
+    q_d = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).to(dev)
+    w_d = torch.from_numpy(w).to(dev)
+    vl_d = torch.from_numpy(vl).to(dev)
+    kcb = kc.nbytes
+    Rk = max(3, -(-2 * L2_BYTES // kcb) + 1)
+    kcs = [torch.from_numpy(kc.view(np.int16)).view(torch.bfloat16).to(dev) for _ in range(Rk)]
+    B, n = x_host.shape
+    k1, k2 = SAMPLING["ks"]
+    idx1 = torch.empty((B, k1), dtype=torch.int32, device=dev)
+    val1 = torch.empty((B, k1), dtype=torch.float32, device=dev)
+    idx2 = torch.empty((B, k2), dtype=torch.int32, device=dev)
+    val2 = torch.empty((B, k2), dtype=torch.float32, device=dev)
+    didx = torch.empty((DECODE["batch"], DECODE["k"]), dtype=torch.int32, device=dev)
+
+    # Each phase of a step is captured G times in a CUDA graph (one replay =
+    # G calls, inputs rotating), so host launch overhead stays off the device
+    # timeline.  A step is one call of each phase.
+    def phase_a(i):
+        ds.ds_topk(xs[i % R], k1, return_value=True, out_idx=idx1, out_val=val1)
+
+    def phase_b(i):
+        ds.ds_topk(xs2[i % R], k2, return_value=True, out_idx=idx2, out_val=val2)
+
+    def phase_c(i):
+        ds.ds_indexer_topk(q_d, kcs[i % Rk], w_d, DECODE["k"], valid_len=vl_d, out_idx=didx)
+
+    phases = (phase_a, phase_b, phase_c)
+    for i in range(args.warmup):
+        for ph in phases:
+            ph(i)
+    torch.cuda.synchronize()
+    status = ds.ds_get_device_status()
+    if status != ds.DS_OK:
+        raise RuntimeError(f"device status after warm-up: {ds.strerror(status)}")
+
+    G = min(args.steps, 200)
+    chunks = [G] * (args.steps // G) + ([args.steps % G] if args.steps % G else [])
+
+    def capture(ph, count, first):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(count):
+                ph(first + i)
+        return g
+
+    graphs = {}
+    for c in sorted(set(chunks)):
+        graphs[c] = [capture(ph, c, 0) for ph in phases]
+    for c in graphs:                       # warm the graphs once
+        for g in graphs[c]:
+            g.replay()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(gpu_uuid(dev))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in chunks]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    t_start.record(stream)
+    for ci, c in enumerate(chunks):
+        ga, gb, gc = graphs[c]
+        evs[ci][0].record(stream)
+        ga.replay()
+        evs[ci][1].record(stream)
+        gb.replay()
+        evs[ci][2].record(stream)
+        gc.replay()
+        evs[ci][3].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    sampler.stop()
+    barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    ph_ms = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])] for e in evs])
+    t_k1, t_k2, t_dec = (ph_ms.sum(axis=0) / args.steps).tolist()        # ms per call
+    total_ms, t_k1, t_k2, t_dec = max_over_ranks([total_ms, t_k1, t_k2, t_dec], dev)
+    status = ds.ds_get_device_status()
+    if status != ds.DS_OK:
+        raise RuntimeError(f"device status after timing: {ds.strerror(status)}")
+
+    b1, b2 = topk_bytes(B, n, k1), topk_bytes(B, n, k2)
+    topk_gbs = ws * (b1 + b2) / ((t_k1 + t_k2) * 1e-3) / 1e9
+    per_launch_gbs = ((b1 + b2) / 2) / (((t_k1 + t_k2) / 2) * 1e-3) / 1e9
+    dbytes, dflops = decode_bytes_flops(vl, DECODE["heads"], DECODE["d"], DECODE["k"])
+    dec_roof_us = max(dbytes / (hbm_gbs * 1e9), dflops / (tflops * 1e12)) * 1e6
+
+    # ---- end to end: pinned host logits in, selection back to host, every step
+    x_pin = torch.from_numpy(x_host).pin_memory()
+    x_dev = torch.empty_like(xs[0])
+    out_pin = [torch.empty((B, k), dtype=torch.int32).pin_memory() for k in (k1, k2)]
+    val_pin = [torch.empty((B, k), dtype=torch.float32).pin_memory() for k in (k1, k2)]
+    e2e_steps = max(3, min(args.steps, 200))
+
+    def e2e_step():
+        x_dev.copy_(x_pin, non_blocking=True)
+        for j, (k, oi, ov) in enumerate(((k1, idx1, val1), (k2, idx2, val2))):
+            ds.ds_topk(x_dev, k, return_value=True, out_idx=oi, out_val=ov)
+            out_pin[j].copy_(oi, non_blocking=True)
+            val_pin[j].copy_(ov, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], dev)
+    e2e_gbs = ws * (b1 + b2) / (e2e_ms * 1e-3) / 1e9
+    h2d = xb
+    d2h = B * (k1 + k2) * 8
+
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "topk_traffic.json")
+    try:
+        import hashlib
+        with open(prof) as f:
+            pj = json.load(f)
+        src = open(os.path.join(ROOT, "sparse_attention_top_ds_b200", "csrc", "topk_kernel.cuh"), "rb").read()
+        if pj.get("kernel_source_sha256") == hashlib.sha256(src).hexdigest():
+            traffic = pj.get("dram_bytes_per_launch")
+    except Exception:
+        traffic = None
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        r = oracle_sample(seconds=10.0)
+        cpu = {"value": round(r["topk_gbs"], 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"{r['topk_rows']} whole sampling rows (k=1024 then 64), single thread; "
+                         f"decode oracle {r['decode_us']:.0f} us/step on {r['decode_rows']} rows"}
+
+    clocks = sampler.summary()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(topk_gbs, 2), "unit": "GB/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": "sampling top-k 64x129280 f32 (N(0,9) + 20 planted +15/row), k=1024 and k=64, "
+                                   "values+indices, unsorted; plus decode indexer+top-k 8x64x128 bf16 vs 32768 "
+                                   "bf16 keys, valid_len~U{4096..32768}, k=1024",
+                       "global_batch": ws * B, "seq_len": n, "parallelism": f"replicas{ws}",
+                       "l2": f"inputs rotate through 2x{R} logit copies and {Rk} key caches (> 2x L2 between reuses)"},
+            "topk_pct_of_peak": round(100 * per_launch_gbs / hbm_gbs, 1),
+            "topk_us_per_call": {"k1024": round(t_k1 * 1e3, 2), "k64": round(t_k2 * 1e3, 2)},
+            "decode_us_per_step": round(t_dec * 1e3, 2),
+            "decode_roofline_us": round(dec_roof_us, 3),
+            "decode_frac_of_roofline": round(dec_roof_us / (t_dec * 1e3), 3),
+            "roofline": {"bound": "hbm", "achieved": round(per_launch_gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": round(per_launch_gbs / hbm_gbs, 4), "traffic": traffic,
+                         "kernel": "topk_cluster_kernel<F32Keys>", "peak_source": peak_src},
+            "e2e": {"value": round(e2e_gbs, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

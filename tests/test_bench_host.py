@@ -1,0 +1,69 @@
+"""Host-side logic of bench.py (CPU only): algorithmic byte / FLOP counts, the
+clock-log summary, and the max-over-ranks reduction with two gloo ranks."""
+
+import os
+import socket
+
+import numpy as np
+import torch.multiprocessing as mp
+
+import bench
+
+
+def test_topk_bytes():
+    # 64 rows x 129280 float32 read once; k (index + value) written per row
+    assert bench.topk_bytes(64, 129280, 1024) == 64 * 129280 * 4 + 64 * 1024 * 8
+    assert bench.topk_bytes(4, 8192, 512, elem=2) == 4 * 8192 * 2 + 4 * 512 * 6
+
+
+def test_decode_bytes_and_flops():
+    vl = np.array([4096, 32768, 10000], dtype=np.int32)
+    b, f = bench.decode_bytes_flops(vl, 64, 128, 1024)
+    assert f == 2 * 64 * 128 * int(vl.sum())
+    assert b == 32768 * 256 + 3 * 64 * 128 * 2 + 3 * 64 * 4 + 3 * 4 + 3 * 1024 * 4
+
+
+def test_clock_summary_flags_throttle_reasons():
+    s = bench.ClockSampler(None)
+    s.lines = [
+        "0, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "0, 1800, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1700, 1965, 995.0, 0x4, Not Active, Not Active, Not Active, Active",
+    ]
+    out = s.summary()
+    assert out["sm_mhz"] == 1800 and out["sm_max_mhz"] == 1965
+    assert out["reasons"] == ["sw_power_cap"] and out["samples"] == 3
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    r, ws = bench.dist_setup("gloo")
+    got = bench.max_over_ranks([float(rank + 1), 10.0 - rank], "cpu")
+    bench.barrier()
+    import torch.distributed as dist
+    dist.destroy_process_group()
+    q.put((r, ws, got))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def test_max_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r, ws, got in res:
+        assert ws == 2
+        assert got == [2.0, 10.0]
