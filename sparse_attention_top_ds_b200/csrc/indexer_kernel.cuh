@@ -46,7 +46,12 @@ struct ScoreCfg {
   static constexpr int kN = NT * HP;                 // accumulator columns per tile
   static constexpr int kNmma = kN < 256 ? kN : 256;  // N of one MMA instruction
   static constexpr int kNumMma = kN / kNmma;
-  static constexpr int kNbuf = kN <= 256 ? 2 : 1;    // TMEM accumulator buffers
+  static constexpr int kNbuf = kN <= 256 ? 2 : 1;    // TMEM accumulator buffers (per tile)
+  // kN == 512 (8 rows x 64 heads): the accumulator is split into two halves of
+  // 256 columns with their own barriers, so the epilogue of one half overlaps
+  // the MMAs of the other; otherwise whole tiles alternate between 2 buffers.
+  static constexpr bool kSplit = (kN == 512);
+  static constexpr int kEpiPerSlot = kSplit ? 4 : 8;  // epilogue warps releasing one accumulator slot
   static constexpr int kCols = kN * kNbuf;
   static constexpr int kTmemCols = kCols <= 32 ? 32 : (kCols <= 64 ? 64 : (kCols <= 128 ? 128 : (kCols <= 256 ? 256 : 512)));
   static constexpr int kQHalf = kN * 128;            // bytes: kN rows x 64 channels x 2 B
@@ -113,11 +118,21 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(BAR(C::kBarAFull + b), 1);
-      mbar_init(BAR(C::kBarAEmpty + b), C::kEpiWarps);
+      mbar_init(BAR(C::kBarAEmpty + b), C::kEpiPerSlot);
     }
     fence_mbar_init();
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
+    // start the loads at once: the queries and the first ring of key tiles
+    if (nact > 0) {
+      mbar_arrive_expect_tx(BAR(C::kBarQ), 2 * C::kQHalf);
+      tma_load_3d(sbase + C::kOffQ, &tm_q, 0, 0, t0, BAR(C::kBarQ));
+      tma_load_3d(sbase + C::kOffQ + C::kQHalf, &tm_q, 64, 0, t0, BAR(C::kBarQ));
+      for (int i = 0; i < min(nact, STAGES); ++i) {
+        const int pos0 = (tile_lo + i) * 128;
+        mbar_arrive_expect_tx(BAR(C::kBarKFull + i), C::kStage);
+        tma_load_2d(sbase + C::kOffK + i * C::kStage, &tm_k, 0, pos0, BAR(C::kBarKFull + i));
+        tma_load_2d(sbase + C::kOffK + i * C::kStage + C::kKHalf, &tm_k, 64, pos0, BAR(C::kBarKFull + i));
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
@@ -136,10 +151,7 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
   if (warp == 0) {
     // ---------------- TMA producer
     if (lane == 0 && nact > 0) {
-      mbar_arrive_expect_tx(BAR(C::kBarQ), 2 * C::kQHalf);
-      tma_load_3d(sbase + C::kOffQ, &tm_q, 0, 0, t0, BAR(C::kBarQ));
-      tma_load_3d(sbase + C::kOffQ + C::kQHalf, &tm_q, 64, 0, t0, BAR(C::kBarQ));
-      for (int i = 0; i < nact; ++i) {
+      for (int i = STAGES; i < nact; ++i) {
         const int s = i % STAGES, r = i / STAGES;
         if (!mbar_wait_bounded(BAR(C::kBarKEmpty + s), (r & 1) ^ 1, p.status)) break;
         const int pos0 = (tile_lo + i) * 128;
@@ -155,27 +167,38 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
       bool ok = mbar_wait_bounded(BAR(C::kBarQ), 0, p.status);
       for (int i = 0; i < nact && ok; ++i) {
         const int s = i % STAGES, r = i / STAGES;
-        const int b = i % C::kNbuf, u = i / C::kNbuf;
-        if (!mbar_wait_bounded(BAR(C::kBarAEmpty + b), (u & 1) ^ 1, p.status)) break;
         if (!mbar_wait_bounded(BAR(C::kBarKFull + s), r & 1, p.status)) break;
-        tc_fence_after();
         const uint32_t a_base = sbase + C::kOffK + s * C::kStage;
-        const uint32_t d_base = tmem_base + (uint32_t)(b * C::kN);
+        // one accumulator slot per MMA group: the two halves (split mode) or
+        // the whole tile in buffer i % 2
+        constexpr int kGroups = C::kSplit ? 2 : 1;
+        constexpr int kMmaPerGroup = C::kNumMma / kGroups;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (uint32_t)(kk & 3) * 32u;  // 16 channels = 32 bytes inside the swizzled row
-          const uint32_t a_addr = a_base + (uint32_t)(kk >> 2) * C::kKHalf + koff;
-          const uint64_t adesc = sw128_kmajor_desc(a_addr);
-#pragma unroll
-          for (int j = 0; j < C::kNumMma; ++j) {
-            const uint32_t b_addr = sbase + C::kOffQ + (uint32_t)(kk >> 2) * C::kQHalf +
-                                    (uint32_t)(j * C::kNmma) * 128u + koff;
-            mma_bf16_ss(d_base + (uint32_t)(j * C::kNmma), adesc, sw128_kmajor_desc(b_addr), idesc,
-                        kk > 0 ? 1u : 0u);
+        for (int g = 0; g < kGroups; ++g) {
+          const int slot = C::kSplit ? g : (i % C::kNbuf);
+          const int use = C::kSplit ? i : (i / C::kNbuf);
+          if (!mbar_wait_bounded(BAR(C::kBarAEmpty + slot), (use & 1) ^ 1, p.status)) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          const uint32_t d_base = tmem_base + (uint32_t)((C::kSplit ? 0 : slot) * C::kN);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t koff = (uint32_t)(kk & 3) * 32u;  // 16 channels = 32 bytes inside the swizzled row
+            const uint64_t adesc = sw128_kmajor_desc(a_base + (uint32_t)(kk >> 2) * C::kKHalf + koff);
+#pragma unroll
+            for (int jj = 0; jj < kMmaPerGroup; ++jj) {
+              const int j = g * kMmaPerGroup + jj;
+              const uint32_t b_addr = sbase + C::kOffQ + (uint32_t)(kk >> 2) * C::kQHalf +
+                                      (uint32_t)(j * C::kNmma) * 128u + koff;
+              mma_bf16_ss(d_base + (uint32_t)(j * C::kNmma), adesc, sw128_kmajor_desc(b_addr), idesc,
+                          kk > 0 ? 1u : 0u);
+            }
+          }
+          mma_commit(BAR(C::kBarAFull + slot));
         }
         mma_commit(BAR(C::kBarKEmpty + s));
-        mma_commit(BAR(C::kBarAFull + b));
       }
     }
   } else {
@@ -199,8 +222,10 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
       vl[j] = v;
     }
     for (int i = 0; i < nact; ++i) {
-      const int b = i % C::kNbuf, u = i / C::kNbuf;
-      if (!mbar_wait_bounded(BAR(C::kBarAFull + b), u & 1, p.status)) break;  // status records the timeout
+      const int b = C::kSplit ? 0 : (i % C::kNbuf);   // TMEM buffer of this tile
+      const int slot = C::kSplit ? hf : b;             // accumulator slot this warp waits on
+      const int u = C::kSplit ? i : (i / C::kNbuf);
+      if (!mbar_wait_bounded(BAR(C::kBarAFull + slot), u & 1, p.status)) break;  // status records the timeout
       tc_fence_after();
       const int s = (tile_lo + i) * 128 + row;
 #pragma unroll
@@ -220,7 +245,7 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C::kBarAEmpty + b));
+      if (lane == 0) mbar_arrive(BAR(C::kBarAEmpty + slot));
     }
     // tiles past the group's valid lengths: no products, -inf
     for (int tile = act_hi > tile_lo ? act_hi : tile_lo; tile < tile_hi; ++tile) {

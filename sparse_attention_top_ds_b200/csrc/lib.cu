@@ -125,7 +125,8 @@ static cudaError_t launch_topk(const TopkParams& p, int C, cudaStream_t st) {
 }
 
 static int topk_enqueue(const void* scores, int batch, int n, int k, int dtype, const int32_t* valid_len,
-                        int32_t* out_idx, void* out_val, int return_value, cudaStream_t st, DeviceState* s) {
+                        int32_t* out_idx, void* out_val, int return_value, int sorted_index, cudaStream_t st,
+                        DeviceState* s) {
   const int elem = dtype == DS_F32 ? 4 : 2;
   TopkShape sh;
   if (!choose_topk_shape(batch, n, elem, s->num_sms, &sh)) return DS_ERR_ARG;
@@ -140,6 +141,7 @@ static int topk_enqueue(const void* scores, int batch, int n, int k, int dtype, 
   p.k = k;
   p.slice = sh.slice;
   p.return_value = return_value ? 1 : 0;
+  p.sorted = sorted_index ? 1 : 0;
   cudaError_t e;
   if (dtype == DS_F32)
     e = sh.threads == 512 ? launch_topk<F32Keys, 512>(p, sh.cluster, st) : launch_topk<F32Keys, 256>(p, sh.cluster, st);
@@ -277,11 +279,10 @@ extern "C" int ds_topk(const void* scores, int batch, int n, int k, int dtype, c
   if (return_value && !out_val) return DS_ERR_ARG;
   if ((long)n * (dtype == DS_F32 ? 4 : 2) > 8L * kMaxSliceBytes) return DS_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(scores) & (dtype == DS_F32 ? 3u : 1u)) != 0) return DS_ERR_ARG;
-  (void)sorted_index;  // the selection is always written in ascending position order
   DeviceState* s = nullptr;
   const int rc = device_state(&s);
   if (rc != DS_OK) return rc;
-  return topk_enqueue(scores, batch, n, k, dtype, valid_len, out_idx, out_val, return_value,
+  return topk_enqueue(scores, batch, n, k, dtype, valid_len, out_idx, out_val, return_value, sorted_index,
                       static_cast<cudaStream_t>(stream), s);
 }
 
@@ -348,5 +349,5 @@ extern "C" int ds_indexer_topk(const void* q, const void* kcache, const float* w
   if (!scores) return DS_ERR_NOMEM;
   rc = score_enqueue(q, kcache, w, batch, heads, S, valid_len, scores, st, s);
   if (rc != DS_OK) return rc;
-  return topk_enqueue(scores, batch, S, k, DS_F32, valid_len, out_idx, out_score, out_score != nullptr, st, s);
+  return topk_enqueue(scores, batch, S, k, DS_F32, valid_len, out_idx, out_score, out_score != nullptr, 0, st, s);
 }

@@ -3,25 +3,26 @@
 // What it computes: for each row, the k largest of the first L = valid_len
 // scores, ties to the lower position (DeepSelect hub page, use-case
 // paragraphs: top-k of a bfloat16 indexer score row, and of a float32 logit
-// row over a ~129K vocabulary).  The selection is returned in ascending
-// position order, so the sorted_index option costs nothing.
+// row over a ~129K vocabulary; options sorted_index and return_value).
 //
 // How (B200 design, not the pages' design):
 //  * A row is split into C contiguous slices, one per CTA of a cluster of C
 //    CTAs.  Each CTA pulls its slice into shared memory with bulk TMA copies
 //    (the row is read from HBM exactly once) and turns every score into an
-//    order-preserving unsigned key in place.
-//  * The k-th largest key is found MSB-first, one radix digit per pass
-//    (float32: 11+11+10 bits, bfloat16: 11+5 bits).  Each CTA builds a local
-//    digit histogram in shared memory; the histograms are added into the
-//    leader CTA through distributed shared memory; the leader finds the digit
-//    holding the k-th key and every CTA reads it back.  A pass stops early
-//    when the whole digit bin is selected.
-//  * Selection count per CTA = keys above the threshold + its share of the
-//    ties, the ties going to the lowest positions of the row (CTA order =
-//    position order).  One ordered pass per CTA (warp scans + a block scan
-//    per chunk) writes indices, and values re-read bit-exactly from global
-//    memory, at ascending output slots.
+//    order-preserving unsigned key in place, building the histogram of the
+//    first radix digit (11 bits) as the chunks land.
+//  * The histograms are added into the leader CTA through distributed shared
+//    memory; the leader finds the digit bin holding the k-th key and every CTA
+//    reads it back.  One more pass over the slice moves the keys above that bin
+//    to a selection list and the keys inside it to a small candidate list; the
+//    remaining digits (float32: 11 + 10 bits, bfloat16: 5 bits) are resolved on
+//    the candidate lists only.  A CTA whose share of the bin overflows its list
+//    scans its whole slice instead (same result, slower).
+//  * Output slots: keys above the threshold, then ties, the ties going to the
+//    lowest positions of the row (CTA order = position order).  With
+//    sorted_index the selection is written by an ordered pass over the slice
+//    (warp scans + a block scan per chunk) and so comes out in ascending
+//    position order.  Values are re-read bit-exactly from global memory.
 #pragma once
 
 #include "ptx.cuh"
@@ -37,6 +38,7 @@ struct TopkParams {
   int batch, n, k;
   int slice;  // elements per CTA, a multiple of 8
   int return_value;
+  int sorted;  // write the selection in ascending position order
 };
 
 // float32 rows: 32-bit keys, digits of 11, 11 and 10 bits.
@@ -86,7 +88,9 @@ struct BF16Keys {
 constexpr int kHistBins = 2048;        // largest digit: 11 bits
 constexpr int kChunkBytes = 16384;     // one TMA copy / mbarrier per 16 KiB
 constexpr int kMaxChunks = 16;
-constexpr int kMaxSliceBytes = 196608; // 192 KiB of scores per CTA
+constexpr int kMaxSliceBytes = 184320; // 180 KiB of scores per CTA
+constexpr int kSelCap = 2048;          // keys above the first-digit bin (< k <= 2048)
+constexpr int kCandCap = 1024;         // keys inside the first-digit bin, per CTA
 
 struct TopkCtrl {
   uint32_t bstar;     // leader -> all: digit of the k-th key in this pass
@@ -98,14 +102,23 @@ struct TopkCtrl {
   uint32_t base;      // this CTA: first output slot
   uint32_t take;      // this CTA: ties it selects
   uint32_t bcast[4];  // broadcast scratch inside the CTA
+  uint32_t sel_cnt;   // entries in the selection list
+  uint32_t cand_cnt;  // entries in the candidate list
+  uint32_t tie_cnt;   // entries in the tie list
+  uint32_t out_cnt;   // output slots handed out (list mode)
 };
 
 constexpr int kSmemHist = 0;
 constexpr int kSmemHred = kSmemHist + kHistBins * 4;
 constexpr int kSmemCtrl = kSmemHred + kHistBins * 4;
-constexpr int kSmemWtot = kSmemCtrl + 64;
+constexpr int kSmemWtot = kSmemCtrl + 128;
 constexpr int kSmemMbar = kSmemWtot + 32 * 4;
-constexpr int kSmemData = ((kSmemMbar + kMaxChunks * 8) + 127) / 128 * 128;
+constexpr int kSmemSel = kSmemMbar + kMaxChunks * 8;
+constexpr int kSmemCandKey = kSmemSel + kSelCap * 4;
+constexpr int kSmemCandIdx = kSmemCandKey + kCandCap * 4;
+constexpr int kSmemTie = kSmemCandIdx + kCandCap * 4;
+constexpr int kSmemData = ((kSmemTie + kCandCap * 4) + 127) / 128 * 128;
+static_assert(sizeof(TopkCtrl) <= 128, "ctrl block");
 
 __host__ __device__ constexpr int topk_smem_bytes(int slice_bytes) { return kSmemData + slice_bytes + 32; }
 
@@ -210,6 +223,10 @@ __global__ void __launch_bounds__(NT, 1) topk_cluster_kernel(const TopkParams p)
   if (tid == 0) {
     for (int j = 0; j < nchunks; ++j) mbar_init(mbar0 + 8 * j, 1);
     fence_mbar_init();
+    ctrl->sel_cnt = 0u;
+    ctrl->cand_cnt = 0u;
+    ctrl->tie_cnt = 0u;
+    ctrl->out_cnt = 0u;
   }
   // The (at most two) words that the slice covers only in part are loaded
   // element by element; their other slots are never read as keys.
@@ -285,39 +302,54 @@ __global__ void __launch_bounds__(NT, 1) topk_cluster_kernel(const TopkParams p)
   cluster_wait();
 
   // ---- radix passes
+  uint32_t* sel_idx = reinterpret_cast<uint32_t*>(smem + kSmemSel);
+  uint32_t* cand_key = reinterpret_cast<uint32_t*>(smem + kSmemCandKey);
+  uint32_t* cand_idx = reinterpret_cast<uint32_t*>(smem + kSmemCandIdx);
+  uint32_t* tie_idx = reinterpret_cast<uint32_t*>(smem + kSmemTie);
   const uint32_t leader_hred = dsmem_map(smem_u32(hred), 0);
   const uint32_t leader_ctrl = dsmem_map(smem_u32(ctrl), 0);
   int krem = kk;
   uint32_t prefix = 0;
   int lvl_shift = 0;
   uint32_t gt_local = 0, eq_local = 0;
+  bool use_list = false;  // per CTA: later digits resolved on the candidate list
+
+  auto elem_of = [&](int w, int j) -> int { return (16 * w + j * K::kBytes - (int)off) / K::kBytes; };
 
   for (int pass = 0; pass < K::kPasses; ++pass) {
     const int sh = K::shift(pass);
     const int nb = 1 << K::width(pass);
     if (pass > 0) {
       const int psh = K::shift(pass - 1);
-      for (int w = tid; w < nwords; w += NT) {
-        const uint4 v = lds128(data + 16 * w);
-        const bool full = (w >= wf0 && w < wf1);
-        uint32_t b0 = 0xFFFFFFFFu;
-        bool same = full;
-#pragma unroll
-        for (int j = 0; j < K::kVec; ++j) {
-          const uint32_t kv = K::slot(v, j);
-          const bool hit = (full || word_valid(w, j)) && (kv >> psh) == prefix;
-          const uint32_t b = hit ? ((kv >> sh) & (uint32_t)(nb - 1)) : 0xFFFFFFFEu;
-          if (j == 0) b0 = b;
-          same &= (b == b0) && hit;
+      if (use_list) {
+        const int nc = min((int)ctrl->cand_cnt, kCandCap);
+        for (int i = tid; i < nc; i += NT) {
+          const uint32_t kv = cand_key[i];
+          if ((kv >> psh) == prefix) atomicAdd(hist + ((kv >> sh) & (uint32_t)(nb - 1)), 1u);
         }
-        if (same) {
-          hist_add_run(hist, b0, K::kVec);
-        } else {
+      } else {
+        for (int w = tid; w < nwords; w += NT) {
+          const uint4 v = lds128(data + 16 * w);
+          const bool full = (w >= wf0 && w < wf1);
+          uint32_t b0 = 0xFFFFFFFFu;
+          bool same = full;
 #pragma unroll
           for (int j = 0; j < K::kVec; ++j) {
             const uint32_t kv = K::slot(v, j);
-            if ((full || word_valid(w, j)) && (kv >> psh) == prefix)
-              atomicAdd(hist + ((kv >> sh) & (uint32_t)(nb - 1)), 1u);
+            const bool hit = (full || word_valid(w, j)) && (kv >> psh) == prefix;
+            const uint32_t b = hit ? ((kv >> sh) & (uint32_t)(nb - 1)) : 0xFFFFFFFEu;
+            if (j == 0) b0 = b;
+            same &= (b == b0) && hit;
+          }
+          if (same) {
+            hist_add_run(hist, b0, K::kVec);
+          } else {
+#pragma unroll
+            for (int j = 0; j < K::kVec; ++j) {
+              const uint32_t kv = K::slot(v, j);
+              if ((full || word_valid(w, j)) && (kv >> psh) == prefix)
+                atomicAdd(hist + ((kv >> sh) & (uint32_t)(nb - 1)), 1u);
+            }
           }
         }
       }
@@ -377,8 +409,36 @@ __global__ void __launch_bounds__(NT, 1) topk_cluster_kernel(const TopkParams p)
     lvl_shift = sh;
     __syncthreads();
     for (int b = tid; b < nb; b += NT) hist[b] = 0u;
-    if (bcount == (uint32_t)krem) break;  // the whole digit bin is selected: threshold found
+    if (pass == 0) {
+      // keys above the bin go to the selection list, keys inside it to the
+      // candidate list (when this CTA's share fits)
+      use_list = eq_local <= (uint32_t)kCandCap;
+      if (use_list) {
+        for (int w = tid; w < nwords; w += NT) {
+          const uint4 v = lds128(data + 16 * w);
+          const bool full = (w >= wf0 && w < wf1);
+#pragma unroll
+          for (int j = 0; j < K::kVec; ++j) {
+            const uint32_t kv = K::slot(v, j);
+            const uint32_t d = kv >> sh;
+            if (d >= prefix && (full || word_valid(w, j))) {
+              if (d > prefix) {
+                const uint32_t pos = atomicAdd(&ctrl->sel_cnt, 1u);
+                if (pos < (uint32_t)kSelCap) sel_idx[pos] = (uint32_t)elem_of(w, j);
+              } else {
+                const uint32_t pos = atomicAdd(&ctrl->cand_cnt, 1u);
+                if (pos < (uint32_t)kCandCap) {
+                  cand_key[pos] = kv;
+                  cand_idx[pos] = (uint32_t)elem_of(w, j);
+                }
+              }
+            }
+          }
+        }
+      }
+    }
     __syncthreads();
+    if (bcount == (uint32_t)krem) break;  // the whole digit bin is selected: threshold found
   }
 
   // ---- exchange (gt, eq) across the cluster; derive output base and tie share
@@ -403,10 +463,17 @@ __global__ void __launch_bounds__(NT, 1) topk_cluster_kernel(const TopkParams p)
   __syncthreads();
   cluster_arrive();  // this CTA no longer reads other CTAs' shared memory
 
-  // ---- ordered emission
   const uint32_t base = ctrl->base, take = ctrl->take;
   const uint32_t mine = gt_local + take;
-  if (mine > 0) {
+  auto put = [&](uint32_t pos, int e_idx) {
+    if (pos < (uint32_t)kk) {  // always true when the counts are consistent
+      out_idx[pos] = i0 + e_idx;
+      if (out_val) out_val[pos] = grow[i0 + e_idx];
+    }
+  };
+
+  if (mine > 0 && (p.sorted || !use_list)) {
+    // ---- ordered emission over the whole slice (ascending positions)
     uint32_t gt_run = 0, tie_run = 0;
     for (int w0 = 0; w0 < nwords; w0 += NT) {
       const int w = w0 + tid;
@@ -434,14 +501,7 @@ __global__ void __launch_bounds__(NT, 1) topk_cluster_kernel(const TopkParams p)
 #pragma unroll
         for (int j = 0; j < K::kVec; ++j) {
           const bool isg = (gm >> j) & 1u, ise = (em >> j) & 1u;
-          if (isg || (ise && tb < take)) {
-            const uint32_t pos = base + gb + min(tb, take);
-            const int e_idx = (16 * w + j * K::kBytes - (int)off) / K::kBytes;
-            if (pos < (uint32_t)kk) {  // always true when the counts are consistent
-              out_idx[pos] = i0 + e_idx;
-              if (out_val) out_val[pos] = grow[i0 + e_idx];
-            }
-          }
+          if (isg || (ise && tb < take)) put(base + gb + min(tb, take), elem_of(w, j));
           gb += isg;
           tb += ise;
         }
@@ -449,6 +509,33 @@ __global__ void __launch_bounds__(NT, 1) topk_cluster_kernel(const TopkParams p)
       gt_run += total & 0xFFFFu;
       tie_run += total >> 16;
       if (gt_run + min(tie_run, take) >= mine) break;  // uniform: every selected key is written
+    }
+  } else if (mine > 0) {
+    // ---- list emission: selection list, then candidates above / at the threshold
+    const int ns = min((int)ctrl->sel_cnt, kSelCap);
+    for (int i = tid; i < ns; i += NT) put(base + atomicAdd(&ctrl->out_cnt, 1u), (int)sel_idx[i]);
+    const int nc = min((int)ctrl->cand_cnt, kCandCap);
+    for (int i = tid; i < nc; i += NT) {
+      const uint32_t top = cand_key[i] >> lvl_shift;
+      if (top > prefix) {
+        put(base + atomicAdd(&ctrl->out_cnt, 1u), (int)cand_idx[i]);
+      } else if (top == prefix && take > 0) {
+        const uint32_t t = atomicAdd(&ctrl->tie_cnt, 1u);
+        tie_idx[t] = cand_idx[i];
+      }
+    }
+    __syncthreads();
+    const int nt = (int)ctrl->tie_cnt;
+    if (take >= (uint32_t)nt) {
+      for (int i = tid; i < nt; i += NT) put(base + gt_local + (uint32_t)i, (int)tie_idx[i]);
+    } else {
+      // the `take` lowest positions among this CTA's ties
+      for (int i = tid; i < nt; i += NT) {
+        const uint32_t me = tie_idx[i];
+        uint32_t rank = 0;
+        for (int j = 0; j < nt; ++j) rank += tie_idx[j] < me;
+        if (rank < take) put(base + gt_local + rank, (int)me);
+      }
     }
   }
   cluster_wait();  // keep this CTA's shared memory alive until the cluster is done reading it

@@ -169,9 +169,9 @@ def test_many_short_rows(cuda_device):
 
 def test_longest_rows(cuda_device):
     g = np.random.default_rng(7)
-    x = g.standard_normal((2, 393216), dtype=np.float32)
+    x = g.standard_normal((2, 368640), dtype=np.float32)
     run_case(x, "f32", 2048)
-    run_case(inputs.f32_to_bf16_bits(g.standard_normal((2, 786432), dtype=np.float32)), "bf16", 2048)
+    run_case(inputs.f32_to_bf16_bits(g.standard_normal((2, 737280), dtype=np.float32)), "bf16", 2048)
 
 
 @pytest.mark.parametrize("cluster", ["1", "2", "4", "8"])
@@ -190,6 +190,6 @@ def test_argument_errors(cuda_device):
         ds.ds_topk(x, 0)
     with pytest.raises(ds.DsError):
         ds.ds_topk(x, ds.DS_MAX_K + 1)
-    too_long = torch.zeros((1, 393216 + 8), dtype=torch.float32, device="cuda")
+    too_long = torch.zeros((1, 368640 + 8), dtype=torch.float32, device="cuda")
     with pytest.raises(ds.DsError):
         ds.ds_topk(too_long, 10)
