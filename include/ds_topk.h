@@ -137,6 +137,34 @@ int ds_indexer_topk(const void* q, const void* kcache, const float* w,
                     int32_t* out_idx, float* out_score, void* stream);
 
 /*
+ * ds_indexer_topk_noalloc -- ds_indexer_topk for callers that must not
+ * allocate device memory.
+ *   (The pages have no counterpart: this is a deployment variant of the same
+ *    computation.)
+ *
+ * Some callers cannot call cudaMalloc: a serving engine that has reserved all
+ * device memory for its own pool, code running while another framework
+ * captures a CUDA graph in a mode that forbids allocation, or a latency-bound
+ * path that cannot take the device-wide synchronisation a first cudaMalloc may
+ * cause.  This entry point never allocates or frees anything: the score rows
+ * go to a fixed 1 MiB array inside the library (held by every GPU that loads
+ * the library until the process exits).
+ *
+ * Arguments, outputs and results are those of ds_indexer_topk, with one more
+ * limit: batch * S <= 262144 (for example 8 rows x 32768 positions); larger
+ * calls return DS_ERR_ARG.
+ * The first call on a device looks up the array's device address (a one-time
+ * set-up with that device current); make that first call before any stream
+ * capture.  Every call on a device uses the same array, which keeps the last
+ * call's contents: calls that overlap on the GPU (different streams, no
+ * ordering between them) race with each other, so order them on one stream.
+ */
+int ds_indexer_topk_noalloc(const void* q, const void* kcache, const float* w,
+                            int batch, int heads, int d, int S,
+                            const int32_t* valid_len, int k,
+                            int32_t* out_idx, float* out_score, void* stream);
+
+/*
  * ds_get_device_status -- synchronise `stream`, then return and clear the
  * current device's status word: DS_OK, or DS_ERR_TIMEOUT if a kernel's bounded
  * wait ran out since the last call (its outputs are then unspecified), or

@@ -55,6 +55,8 @@ def load():
     lib.ds_indexer_score.restype = i32
     lib.ds_indexer_topk.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32p, i32, vp, vp, vp]
     lib.ds_indexer_topk.restype = i32
+    lib.ds_indexer_topk_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32p, i32, vp, vp, vp]
+    lib.ds_indexer_topk_noalloc.restype = i32
     lib.ds_get_device_status.argtypes = [vp]
     lib.ds_get_device_status.restype = i32
     lib.ds_strerror.argtypes = [i32]
@@ -87,6 +89,12 @@ def ds_indexer_score_raw(q, kcache, w, batch, heads, d, S, valid_len, out_score,
 
 def ds_indexer_topk_raw(q, kcache, w, batch, heads, d, S, valid_len, k, out_idx, out_score, stream):
     return load().ds_indexer_topk(q, kcache, w, batch, heads, d, S, valid_len, k, out_idx, out_score, stream)
+
+
+def ds_indexer_topk_noalloc_raw(q, kcache, w, batch, heads, d, S, valid_len, k, out_idx, out_score, stream):
+    """The allocation-free variant (score rows in the library's fixed array)."""
+    return load().ds_indexer_topk_noalloc(q, kcache, w, batch, heads, d, S, valid_len, k, out_idx, out_score,
+                                          stream)
 
 
 def ds_get_device_status(stream=None):

@@ -351,3 +351,58 @@ extern "C" int ds_indexer_topk(const void* q, const void* kcache, const float* w
   if (rc != DS_OK) return rc;
   return topk_enqueue(scores, batch, S, k, DS_F32, valid_len, out_idx, out_score, out_score != nullptr, 0, st, s);
 }
+
+// ------------------------------------------------------------------ allocation-free indexer + top-k
+//
+// Some callers cannot call cudaMalloc at all: a serving engine that reserves
+// all device memory for its own pool up front, code that runs while another
+// framework is capturing a CUDA graph in a mode that forbids allocation, or a
+// latency-critical path that cannot afford the device-wide synchronisation a
+// first cudaMalloc may cause.  ds_indexer_topk_noalloc serves them: its score
+// rows go to a fixed array in the library's own device memory instead of the
+// grow-only scratch buffer.  Every GPU that loads the library holds this array
+// (1 MiB) until the process exits.
+
+constexpr int kNoAllocScores = 262144;  // floats: batch * S may not exceed this (1 MiB)
+
+// The array itself.  In host code this name is only a host-side stand-in, not
+// a device address; the device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) float g_noalloc_scores[kNoAllocScores];
+
+static float* g_noalloc_ptr[kMaxDevices];  // device address of g_noalloc_scores, per device
+
+// Once per device, with that device current (the first call on the device).
+static int noalloc_scores_ptr(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DS_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scores) != cudaSuccess || !p) return DS_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return DS_OK;
+}
+
+extern "C" int ds_indexer_topk_noalloc(const void* q, const void* kcache, const float* w, int batch, int heads,
+                                       int d, int S, const int32_t* valid_len, int k, int32_t* out_idx,
+                                       float* out_score, void* stream) {
+  int rc = indexer_check(q, kcache, w, batch, heads, d, S);
+  if (rc != DS_OK) return rc;
+  if (!out_idx || k <= 0 || k > DS_MAX_K) return DS_ERR_ARG;
+  if ((long)batch * (long)S > (long)kNoAllocScores) return DS_ERR_ARG;  // beyond the fixed array
+  DeviceState* s = nullptr;
+  rc = device_state(&s);
+  if (rc != DS_OK) return rc;
+  float* scores = nullptr;
+  rc = noalloc_scores_ptr(&scores);
+  if (rc != DS_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The scorer writes every position of every row (-inf at and past
+  // valid_len) before the selection reads it, so nothing left over from an
+  // earlier call is ever read and the array needs no clearing.
+  rc = score_enqueue(q, kcache, w, batch, heads, S, valid_len, scores, st, s);
+  if (rc != DS_OK) return rc;
+  return topk_enqueue(scores, batch, S, k, DS_F32, valid_len, out_idx, out_score, out_score != nullptr, 0, st, s);
+}
