@@ -69,9 +69,7 @@ typedef enum { DS_F32 = 0, DS_BF16 = 1 } ds_dtype;
  *    sampling; options sorted_index and return_value.)
  *
  * scores       device, [batch, n] of `dtype` (float32 or bfloat16), read only.
- * batch, n     rows and row length; batch >= 1, n >= 1, and one row must fit
- *              the on-chip budget: n * sizeof(dtype) <= 1440 KiB
- *              (n <= 368640 float32 or 737280 bfloat16).
+ * batch, n     rows and row length; batch >= 1, 1 <= n <= 16777216.
  * k            1 <= k <= DS_MAX_K.  k may exceed n (extra slots are padding).
  * dtype        DS_F32 or DS_BF16.
  * valid_len    device int32 [batch] or NULL.  Row t considers positions
@@ -123,7 +121,7 @@ int ds_indexer_score(const void* q, const void* kcache, const float* w,
  *
  * q, kcache, w, batch, heads, d, S, valid_len  as for ds_indexer_score.
  * k          1 <= k <= DS_MAX_K.
- * S          additionally S <= 368640 (the selection runs on float32 rows).
+ * S          additionally S <= 16777216.
  * out_idx    device int32 [batch, k]: selected positions, order unspecified,
  *            -1 in padding slots.
  * out_score  device float32 [batch, k] or NULL: the float32 score of each

@@ -35,6 +35,8 @@ static std::mutex g_mu;
 static DeviceState g_dev[kMaxDevices];
 
 static cudaError_t indexer_setup();
+static bool topk_cluster16_ok();
+static int g_max_cluster = 8;  // largest cluster the top-k launch may use
 
 // Set-up once per device, with that device current: capability check, the
 // status word's address, and the kernels' shared-memory limits.
@@ -62,6 +64,7 @@ static int device_state(DeviceState** out) {
         e = cudaFuncSetAttribute(topk_cluster_kernel<BF16Keys, 512>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
       if (e == cudaSuccess) e = indexer_setup();
       if (e != cudaSuccess) return DS_ERR_CUDA;
+      g_max_cluster = topk_cluster16_ok() ? 16 : 8;
     }
     s.ready = true;
   }
@@ -78,32 +81,63 @@ struct TopkShape {
   int threads;   // threads per CTA
 };
 
-// Launch shape: split a row over a cluster until a slice is small enough to
-// sit in shared memory next to other CTAs, and until the grid fills the GPU
-// (about two CTAs per SM), but never below 4 KiB per slice.
-static bool choose_topk_shape(int batch, int n, int elem, int num_sms, TopkShape* out) {
+// Launch shape: a cluster of C CTAs per row (C <= 8, or 16 where the device
+// allows non-portable clusters), enough CTAs to fill every SM several times
+// over, but no slice below 1024 scores.  Shared memory does not hold the
+// scores, so the slice size is free.
+constexpr int kMaxRowElems = 1 << 24;
+
+static bool choose_topk_shape(int batch, int n, int num_sms, TopkShape* out) {
+  if (n > kMaxRowElems) return false;
   int C = 1;
-  const long target = 2L * num_sms;
+  const long target = 4L * num_sms;
   const char* force = getenv("DS_TOPK_CLUSTER");  // tuning sweeps only
   if (force) {
     C = atoi(force);
-    if (C != 1 && C != 2 && C != 4 && C != 8) C = 8;
+    if (C != 1 && C != 2 && C != 4 && C != 8 && C != 16) C = 8;
+    if (C > g_max_cluster) C = g_max_cluster;
   } else {
-    while (C < 8) {
-      const long sb = (long)((n + C - 1) / C) * elem;
-      const bool too_big = sb > 48 * 1024;
-      const bool too_few = (long)batch * C < target && sb > 4096;
-      if (!too_big && !too_few) break;
-      C *= 2;
-    }
+    const int cmax = batch >= 8 ? min(8, g_max_cluster) : g_max_cluster;
+    while (C < cmax && (long)batch * C < target && (n + 2 * C - 1) / (2 * C) >= 1024) C *= 2;
   }
   int slice = (n + C - 1) / C;
   slice = (slice + 7) / 8 * 8;
-  if ((long)slice * elem > kMaxSliceBytes) return false;
   out->cluster = C;
   out->slice = slice;
-  out->threads = ((long)slice * elem >= 32 * 1024) ? 512 : 256;
+  const char* nt = getenv("DS_TOPK_THREADS");      // tuning sweeps only
+  out->threads = (nt && atoi(nt) == 512) ? 512 : 256;
   return true;
+}
+
+// Clusters of 16 CTAs are non-portable: allow them only where the device
+// can run at least one.
+static bool topk_cluster16_ok() {
+  auto kern = topk_cluster_kernel<F32Keys, 256>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  cudaFuncSetAttribute(topk_cluster_kernel<F32Keys, 512>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaFuncSetAttribute(topk_cluster_kernel<BF16Keys, 256>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaFuncSetAttribute(topk_cluster_kernel<BF16Keys, 512>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(16, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)kTopkSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 16;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return n >= 1;
 }
 
 template <class K, int NT>
@@ -112,7 +146,7 @@ static cudaError_t launch_topk(const TopkParams& p, int C, cudaStream_t st) {
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)(p.batch * C), 1, 1);
   cfg.blockDim = dim3(NT, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)topk_smem_bytes(p.slice * K::kBytes);
+  cfg.dynamicSmemBytes = (size_t)kTopkSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -127,9 +161,8 @@ static cudaError_t launch_topk(const TopkParams& p, int C, cudaStream_t st) {
 static int topk_enqueue(const void* scores, int batch, int n, int k, int dtype, const int32_t* valid_len,
                         int32_t* out_idx, void* out_val, int return_value, int sorted_index, cudaStream_t st,
                         DeviceState* s) {
-  const int elem = dtype == DS_F32 ? 4 : 2;
   TopkShape sh;
-  if (!choose_topk_shape(batch, n, elem, s->num_sms, &sh)) return DS_ERR_ARG;
+  if (!choose_topk_shape(batch, n, s->num_sms, &sh)) return DS_ERR_ARG;
   TopkParams p;
   p.scores = scores;
   p.valid_len = valid_len;
@@ -277,7 +310,7 @@ extern "C" int ds_topk(const void* scores, int batch, int n, int k, int dtype, c
   if (!scores || !out_idx || batch <= 0 || n <= 0 || k <= 0 || k > DS_MAX_K) return DS_ERR_ARG;
   if (dtype != DS_F32 && dtype != DS_BF16) return DS_ERR_ARG;
   if (return_value && !out_val) return DS_ERR_ARG;
-  if ((long)n * (dtype == DS_F32 ? 4 : 2) > 8L * kMaxSliceBytes) return DS_ERR_ARG;
+  if (n > kMaxRowElems) return DS_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(scores) & (dtype == DS_F32 ? 3u : 1u)) != 0) return DS_ERR_ARG;
   DeviceState* s = nullptr;
   const int rc = device_state(&s);
@@ -340,7 +373,7 @@ extern "C" int ds_indexer_topk(const void* q, const void* kcache, const float* w
   int rc = indexer_check(q, kcache, w, batch, heads, d, S);
   if (rc != DS_OK) return rc;
   if (!out_idx || k <= 0 || k > DS_MAX_K) return DS_ERR_ARG;
-  if ((long)S * 4 > 8L * kMaxSliceBytes) return DS_ERR_ARG;
+  if (S > kMaxRowElems) return DS_ERR_ARG;
   DeviceState* s = nullptr;
   rc = device_state(&s);
   if (rc != DS_OK) return rc;

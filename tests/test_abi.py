@@ -66,7 +66,7 @@ def test_argument_errors_need_no_gpu(lib):
     assert lib.ds_topk(fake, 1, 10, 2049, 0, None, fake, fake, 1, 0, None) == -1   # k > max
     assert lib.ds_topk(fake, 1, 10, 5, 7, None, fake, fake, 1, 0, None) == -1      # dtype
     assert lib.ds_topk(fake, 1, 10, 5, 0, None, fake, None, 1, 0, None) == -1      # out_val missing
-    assert lib.ds_topk(fake, 1, 400000, 5, 0, None, fake, fake, 1, 0, None) == -1  # row too long
+    assert lib.ds_topk(fake, 1, (1 << 24) + 1, 5, 0, None, fake, fake, 1, 0, None) == -1  # row too long
     assert lib.ds_topk(vp(0x100001), 1, 10, 5, 0, None, fake, fake, 1, 0, None) == -1  # misaligned
     lib.ds_indexer_topk.restype = ctypes.c_int
     lib.ds_indexer_topk.argtypes = [vp, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp,

@@ -167,14 +167,14 @@ def test_many_short_rows(cuda_device):
     run_case(inputs.f32_to_bf16_bits(x), "bf16", 64)
 
 
-def test_longest_rows(cuda_device):
+def test_long_rows(cuda_device):
     g = np.random.default_rng(7)
-    x = g.standard_normal((2, 368640), dtype=np.float32)
+    x = g.standard_normal((2, 1000003), dtype=np.float32)
     run_case(x, "f32", 2048)
-    run_case(inputs.f32_to_bf16_bits(g.standard_normal((2, 737280), dtype=np.float32)), "bf16", 2048)
+    run_case(inputs.f32_to_bf16_bits(g.standard_normal((2, 2000001), dtype=np.float32)), "bf16", 2048)
 
 
-@pytest.mark.parametrize("cluster", ["1", "2", "4", "8"])
+@pytest.mark.parametrize("cluster", ["1", "2", "4", "8", "16"])
 def test_every_cluster_size(cuda_device, cluster, monkeypatch):
     monkeypatch.setenv("DS_TOPK_CLUSTER", cluster)
     g = np.random.default_rng(8)
@@ -190,6 +190,6 @@ def test_argument_errors(cuda_device):
         ds.ds_topk(x, 0)
     with pytest.raises(ds.DsError):
         ds.ds_topk(x, ds.DS_MAX_K + 1)
-    too_long = torch.zeros((1, 368640 + 8), dtype=torch.float32, device="cuda")
+    too_long = torch.zeros((1, (1 << 24) + 8), dtype=torch.float32, device="cuda")
     with pytest.raises(ds.DsError):
         ds.ds_topk(too_long, 10)
