@@ -14,6 +14,7 @@
 #include "ptx.cuh"
 #include "topk_kernel.cuh"
 #include "indexer_kernel.cuh"
+#include "decode_kernel.cuh"
 
 namespace dstopk {
 
@@ -29,6 +30,10 @@ struct DeviceState {
   int* status = nullptr;     // device address of g_status on this device
   void* scratch = nullptr;   // grow-only scratch for ds_indexer_topk
   size_t scratch_bytes = 0;
+  uint32_t* dec_ctl = nullptr;   // fused decode: control table (two copies, zeroed once)
+  uint32_t* dec_cand = nullptr;  // fused decode: candidate lists, grow-only
+  size_t dec_cand_bytes = 0;
+  int dec_max_blocks = 0;        // co-resident CTAs of the fused decode kernel
 };
 
 static std::mutex g_mu;
@@ -210,6 +215,9 @@ static cudaError_t indexer_setup() {
   if (e == cudaSuccess) e = set_score_smem<8, 64, 2>();
   if (e == cudaSuccess) e = set_score_smem<8, 32, 4>();
   if (e == cudaSuccess) e = set_score_smem<8, 16, 4>();
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(indexer_topk_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DecodeSmem::kBytes);
   return e;
 }
 
@@ -273,6 +281,87 @@ static int score_enqueue(const void* q, const void* kc, const float* w, int B, i
   }
   if (H > 16) return launch_score<8, 32, 4>(q, kc, w, B, H, S, vl, out, st, s);
   return launch_score<8, 16, 4>(q, kc, w, B, H, S, vl, out, st, s);
+}
+
+// ---- fused decode (score + top-k in one cooperative launch)
+
+// The single-launch grid-wide variant is opt-in (DS_INDEXER_FUSED=1): on this
+// GPU its chain of grid-wide round trips costs more than the two-kernel path.
+static bool decode_fits(int B, int H, int S, const DeviceState* s) {
+  if (getenv("DS_INDEXER_UNFUSED")) return false;  // testing / comparison only
+  if (!getenv("DS_INDEXER_FUSED")) return false;
+  if (B > kDecRows || H <= 32 || H > kDecHeads) return false;
+  const int ntiles = (S + 127) / 128;
+  return ntiles <= s->num_sms * kDecMaxTiles;
+}
+
+static int decode_enqueue(const void* q, const void* kc, const float* w, int B, int H, int S,
+                          const int32_t* vl, int k, int32_t* out_idx, float* out_score, cudaStream_t st,
+                          DeviceState* s) {
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!s->dec_ctl) {
+      void* p = nullptr;
+      if (cudaMalloc(&p, DecodeCtl::kTotal * sizeof(uint32_t)) != cudaSuccess) {
+        cudaGetLastError();
+        return DS_ERR_NOMEM;
+      }
+      if (cudaMemset(p, 0, DecodeCtl::kTotal * sizeof(uint32_t)) != cudaSuccess) return DS_ERR_CUDA;
+      s->dec_ctl = static_cast<uint32_t*>(p);
+      int per_sm = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, indexer_topk_decode_kernel, kDecThreads,
+                                                        DecodeSmem::kBytes) != cudaSuccess)
+        return DS_ERR_CUDA;
+      s->dec_max_blocks = per_sm * s->num_sms;
+    }
+    const size_t need = (size_t)B * (size_t)S * 2 * sizeof(uint32_t);
+    if (s->dec_cand_bytes < need) {
+      if (s->dec_cand) cudaFree(s->dec_cand);
+      s->dec_cand = nullptr;
+      s->dec_cand_bytes = 0;
+      void* p = nullptr;
+      if (cudaMalloc(&p, need) != cudaSuccess) {
+        cudaGetLastError();
+        return DS_ERR_NOMEM;
+      }
+      s->dec_cand = static_cast<uint32_t*>(p);
+      s->dec_cand_bytes = need;
+    }
+  }
+  const int ntiles = (S + 127) / 128;
+  int G = min(ntiles, min(s->num_sms, s->dec_max_blocks));
+  if (G < 1) return DS_ERR_CUDA;
+  const int tpc = (ntiles + G - 1) / G;
+  if (tpc > kDecMaxTiles) return DS_ERR_ARG;
+  G = (ntiles + tpc - 1) / tpc;
+  CUtensorMap tq, tk;
+  if (!encode_maps(q, kc, B, H, S, kDecHeads, 4, &tq, &tk)) return DS_ERR_ARG;
+  DecodeParams p;
+  p.w = w;
+  p.valid_len = vl;
+  p.out_idx = out_idx;
+  p.out_score = out_score;
+  p.status = s->status;
+  p.B = B;
+  p.H = H;
+  p.S = S;
+  p.k = k;
+  p.tiles_per_cta = tpc;
+  p.ctl = s->dec_ctl;
+  p.cand = s->dec_cand;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)G, 1, 1);
+  cfg.blockDim = dim3(kDecThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)DecodeSmem::kBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, indexer_topk_decode_kernel, tq, tk, p);
+  return e == cudaSuccess ? DS_OK : DS_ERR_CUDA;
 }
 
 static int indexer_check(const void* q, const void* kc, const float* w, int B, int H, int d, int S) {
@@ -348,10 +437,17 @@ extern "C" void ds_release(void) {
   int cur = -1;
   if (cudaGetDevice(&cur) != cudaSuccess) cur = -1;
   for (int d = 0; d < kMaxDevices; ++d) {
-    if (g_dev[d].scratch) {
-      if (cudaSetDevice(d) == cudaSuccess) cudaFree(g_dev[d].scratch);
+    if (g_dev[d].scratch || g_dev[d].dec_ctl || g_dev[d].dec_cand) {
+      if (cudaSetDevice(d) == cudaSuccess) {
+        if (g_dev[d].scratch) cudaFree(g_dev[d].scratch);
+        if (g_dev[d].dec_ctl) cudaFree(g_dev[d].dec_ctl);
+        if (g_dev[d].dec_cand) cudaFree(g_dev[d].dec_cand);
+      }
       g_dev[d].scratch = nullptr;
       g_dev[d].scratch_bytes = 0;
+      g_dev[d].dec_ctl = nullptr;
+      g_dev[d].dec_cand = nullptr;
+      g_dev[d].dec_cand_bytes = 0;
     }
   }
   if (cur >= 0) cudaSetDevice(cur);
@@ -378,6 +474,8 @@ extern "C" int ds_indexer_topk(const void* q, const void* kcache, const float* w
   rc = device_state(&s);
   if (rc != DS_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (decode_fits(batch, heads, S, s))
+    return decode_enqueue(q, kcache, w, batch, heads, S, valid_len, k, out_idx, out_score, st, s);
   float* scores = static_cast<float*>(get_scratch(s, (size_t)batch * (size_t)S * sizeof(float)));
   if (!scores) return DS_ERR_NOMEM;
   rc = score_enqueue(q, kcache, w, batch, heads, S, valid_len, scores, st, s);

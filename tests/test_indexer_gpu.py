@@ -165,3 +165,66 @@ def test_indexer_argument_errors(cuda_device):
     w = torch.zeros((2, 65), dtype=torch.float32, device="cuda")
     with pytest.raises(ds.DsError):
         ds.ds_indexer_topk(q, kc, w, 10)         # heads > 64
+
+
+# ---------------------------------------------------------------- fused decode path
+
+@pytest.fixture
+def grid_fused(monkeypatch):
+    # the single-launch, grid-barrier decode kernel (opt-in)
+    monkeypatch.setenv("DS_INDEXER_FUSED", "1")
+
+
+def test_fused_decode_matches_unfused_path(cuda_device, grid_fused, monkeypatch):
+    # B <= 8 rows and 33..64 heads take the fused single-launch kernel; the
+    # unfused path (scores to scratch, then ds_topk) computes the same float32
+    # scores in the same order, so both select the same positions exactly.
+    q, kc, w, vl = inputs.decode(seed=31)
+    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
+    fused, fs = ds.ds_indexer_topk(qd, kd, wd, 1024, valid_len=vd, return_score=True)
+    torch.cuda.synchronize()
+    monkeypatch.setenv("DS_INDEXER_UNFUSED", "1")
+    ref, rs = ds.ds_indexer_topk(qd, kd, wd, 1024, valid_len=vd, return_score=True)
+    torch.cuda.synchronize()
+    assert ds.ds_get_device_status() == ds.DS_OK
+    f, r = fused.cpu().numpy(), ref.cpu().numpy()
+    for t in range(q.shape[0]):
+        assert np.array_equal(np.sort(f[t]), np.sort(r[t])), f"row {t}"
+        of, orr = np.argsort(f[t]), np.argsort(r[t])
+        assert np.array_equal(fs.cpu().numpy()[t][of], rs.cpu().numpy()[t][orr])
+
+
+@pytest.mark.parametrize("B,S,k", [(1, 40000, 2048), (5, 7000, 512), (8, 128, 64), (2, 75000, 100)])
+def test_fused_decode_shapes(cuda_device, grid_fused, B, S, k):
+    q, kc, w = inputs.indexer_factors(seed=B * 3 + S, batch=B, n=S, heads=64)
+    g = np.random.default_rng(S)
+    vl = g.integers(0, S + 1, size=B).astype(np.int32)
+    vl[0] = S
+    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
+    idx, score = ds.ds_indexer_topk(qd, kd, wd, k, valid_len=vd, return_score=True)
+    torch.cuda.synchronize()
+    assert ds.ds_get_device_status() == ds.DS_OK
+    check_selection(q, kc, w, vl, k, idx.cpu().numpy(), score.cpu().numpy())
+
+
+def test_fused_decode_graph_replay_with_odd_call_count(cuda_device, grid_fused):
+    # the fused kernel alternates between two copies of its control table on
+    # its own; replaying a graph of 3 calls several times must keep results right
+    q, kc, w, vl = inputs.decode(seed=41, S=8192, vl_lo=1000, vl_hi=8192)
+    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
+    outs = [torch.empty((8, 512), dtype=torch.int32, device="cuda") for _ in range(3)]
+    ds.ds_indexer_topk(qd, kd, wd, 512, valid_len=vd, out_idx=outs[0])   # warm-up outside capture
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for o in outs:
+            ds.ds_indexer_topk(qd, kd, wd, 512, valid_len=vd, out_idx=o)
+    ref, _ = oracle.indexer_topk(q, kc, w, 512, vl)
+    for _ in range(3):
+        for o in outs:
+            o.fill_(-7)
+        gr.replay()
+        torch.cuda.synchronize()
+        assert ds.ds_get_device_status() == ds.DS_OK
+        for o in outs:
+            check_selection(q, kc, w, vl, 512, o.cpu().numpy(), None)
