@@ -13,8 +13,10 @@
 #include "../../include/ds_topk.h"
 #include "ptx.cuh"
 #include "topk_kernel.cuh"
+#include "topk_stash_kernel.cuh"
 #include "indexer_kernel.cuh"
 #include "decode_kernel.cuh"
+#include "rowcluster_kernel.cuh"
 
 namespace dstopk {
 
@@ -34,13 +36,23 @@ struct DeviceState {
   uint32_t* dec_cand = nullptr;  // fused decode: candidate lists, grow-only
   size_t dec_cand_bytes = 0;
   int dec_max_blocks = 0;        // co-resident CTAs of the fused decode kernel
+  int rc_cluster = 0;            // row-per-cluster indexer + top-k: CTAs per row (0: unavailable)
+  int rc_active = 0;             // clusters of that size the device runs at once
 };
 
 static std::mutex g_mu;
 static DeviceState g_dev[kMaxDevices];
 
 static cudaError_t indexer_setup();
+template <int NT>
+static cudaError_t set_stash_smem(int bytes) {
+  cudaError_t e = cudaFuncSetAttribute(topk_stash_kernel<F32Keys, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(topk_stash_kernel<BF16Keys, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  return e;
+}
 static bool topk_cluster16_ok();
+static int rowcluster_active(int C);
 static int g_max_cluster = 8;  // largest cluster the top-k launch may use
 
 // Set-up once per device, with that device current: capability check, the
@@ -67,9 +79,16 @@ static int device_state(DeviceState** out) {
         e = cudaFuncSetAttribute(topk_cluster_kernel<BF16Keys, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(topk_cluster_kernel<BF16Keys, 512>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
+      if (e == cudaSuccess) e = set_stash_smem<256>(smem_max);
+      if (e == cudaSuccess) e = set_stash_smem<512>(smem_max);
+      if (e == cudaSuccess) e = set_stash_smem<1024>(smem_max);
       if (e == cudaSuccess) e = indexer_setup();
       if (e != cudaSuccess) return DS_ERR_CUDA;
       g_max_cluster = topk_cluster16_ok() ? 16 : 8;
+      const int a16 = rowcluster_active(16);
+      const int a8 = a16 > 0 ? 0 : rowcluster_active(8);
+      s.rc_cluster = a16 > 0 ? 16 : (a8 > 0 ? 8 : 0);
+      s.rc_active = a16 > 0 ? a16 : a8;
     }
     s.ready = true;
   }
@@ -163,9 +182,79 @@ static cudaError_t launch_topk(const TopkParams& p, int C, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, topk_cluster_kernel<K, NT>, p);
 }
 
+// One-pass stash kernel.  Launch shape: one CTA per row, or C = 2 or 4 CTAs
+// per row (a cluster) while the rows would leave more than half of the SMs
+// idle and every slice keeps at least 32768 scores.
+static int topk_stash_enqueue(const void* scores, int batch, int n, int k, int dtype, const int32_t* valid_len,
+                              int32_t* out_idx, void* out_val, int return_value, int sorted_index,
+                              cudaStream_t st, DeviceState* s) {
+  if (n > kMaxRowElems) return DS_ERR_ARG;
+  int C = 1;
+  const char* force = getenv("DS_TOPK_CLUSTER");  // tuning sweeps only
+  if (force) {
+    C = atoi(force);
+    if (C != 1 && C != 2 && C != 4) C = 1;
+  } else {
+    while (C < kTsMaxCluster && (long)batch * 2 * C <= s->num_sms && n / (2 * C) >= 32768) C *= 2;
+  }
+  int slice = (n + C - 1) / C;
+  slice = (slice + 7) / 8 * 8;
+  TsParams p;
+  p.scores = scores;
+  p.valid_len = valid_len;
+  p.out_idx = out_idx;
+  p.out_val = out_val;
+  p.batch = batch;
+  p.n = n;
+  p.k = k;
+  p.slice = slice;
+  p.return_value = return_value ? 1 : 0;
+  p.sorted = sorted_index ? 1 : 0;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)(batch * C), 1, 1);
+  cfg.blockDim = dim3(kTsThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)ts_smem_bytes(C);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int nt = kTsThreads;
+  const char* fnt = getenv("DS_TOPK_NT");  // tuning sweeps only
+  if (fnt && (atoi(fnt) == 256 || atoi(fnt) == 512 || atoi(fnt) == 1024)) nt = atoi(fnt);
+  cfg.blockDim = dim3((unsigned)nt, 1, 1);
+  cudaError_t e;
+  if (nt == 256)
+    e = dtype == DS_F32 ? cudaLaunchKernelEx(&cfg, topk_stash_kernel<F32Keys, 256>, p)
+                        : cudaLaunchKernelEx(&cfg, topk_stash_kernel<BF16Keys, 256>, p);
+  else if (nt == 1024)
+    e = dtype == DS_F32 ? cudaLaunchKernelEx(&cfg, topk_stash_kernel<F32Keys, 1024>, p)
+                        : cudaLaunchKernelEx(&cfg, topk_stash_kernel<BF16Keys, 1024>, p);
+  else
+    e = dtype == DS_F32 ? cudaLaunchKernelEx(&cfg, topk_stash_kernel<F32Keys, 512>, p)
+                        : cudaLaunchKernelEx(&cfg, topk_stash_kernel<BF16Keys, 512>, p);
+  return e == cudaSuccess ? DS_OK : DS_ERR_CUDA;
+}
+
+// Two kernels: with many rows (>= 32) the one-pass stash kernel, whose rows
+// fill the SMs with one or two CTAs each; with few rows the cluster kernel
+// (topk_kernel.cuh), which spreads a row over up to 16 CTAs and has the
+// shorter fixed chain of steps.  DS_TOPK_KERNEL=stash / cluster picks one
+// regardless (tests and comparisons).
 static int topk_enqueue(const void* scores, int batch, int n, int k, int dtype, const int32_t* valid_len,
                         int32_t* out_idx, void* out_val, int return_value, int sorted_index, cudaStream_t st,
                         DeviceState* s) {
+  bool stash = batch >= 32;
+  const char* pick = getenv("DS_TOPK_KERNEL");
+  if (pick && strcmp(pick, "stash") == 0) stash = true;
+  if (pick && strcmp(pick, "cluster") == 0) stash = false;
+  if (stash)
+    return topk_stash_enqueue(scores, batch, n, k, dtype, valid_len, out_idx, out_val, return_value, sorted_index,
+                              st, s);
   TopkShape sh;
   if (!choose_topk_shape(batch, n, s->num_sms, &sh)) return DS_ERR_ARG;
   TopkParams p;
@@ -218,7 +307,38 @@ static cudaError_t indexer_setup() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(indexer_topk_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              DecodeSmem::kBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(indexer_topk_rowcluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             RcSmem::kBytes);
   return e;
+}
+
+// Clusters the row-per-cluster kernel can run at once with C CTAs each (0 if none).
+static int rowcluster_active(int C) {
+  if (C == 16 &&
+      cudaFuncSetAttribute(indexer_topk_rowcluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)C, 1, 1);
+  cfg.blockDim = dim3(kRcThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)RcSmem::kBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, indexer_topk_rowcluster_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
 }
 
 // bf16 tensor maps with 128-byte swizzle: queries [B][H][128] in boxes of
@@ -364,6 +484,54 @@ static int decode_enqueue(const void* q, const void* kc, const float* w, int B, 
   return e == cudaSuccess ? DS_OK : DS_ERR_CUDA;
 }
 
+// ---- row-per-cluster indexer + top-k (one launch, nothing written but the result)
+
+// Opt-in (DS_INDEXER_ROWCLUSTER=1): with one 16-CTA cluster per row each SM
+// streams 1/16 of the row's keys at the rate one SM reaches alone, and the
+// leader's pass over the row is latency bound, so on this GPU the two-kernel
+// path is faster at every batch size measured (1 to 64 rows).
+static bool rowcluster_fits(int B, int H, int S, const DeviceState* s) {
+  if (s->rc_cluster == 0 || S > kRcMaxS || H > kRcHeads || B <= 0) return false;
+  const char* f = getenv("DS_INDEXER_ROWCLUSTER");
+  return f && atoi(f) == 1;
+}
+
+static int rowcluster_enqueue(const void* q, const void* kc, const float* w, int B, int H, int S,
+                              const int32_t* vl, int k, int32_t* out_idx, float* out_score, cudaStream_t st,
+                              DeviceState* s) {
+  const int C = s->rc_cluster;
+  const int ppc = ((S + C - 1) / C + 127) / 128 * 128;
+  if (ppc > kRcMaxPPC || (long)ppc * C < S) return DS_ERR_ARG;
+  CUtensorMap tq, tk;
+  if (!encode_maps(q, kc, B, H, S, kRcHeads, 1, &tq, &tk)) return DS_ERR_ARG;
+  RowClusterParams p;
+  p.w = w;
+  p.valid_len = vl;
+  p.out_idx = out_idx;
+  p.out_score = out_score;
+  p.status = s->status;
+  p.B = B;
+  p.H = H;
+  p.S = S;
+  p.k = k;
+  p.ppc = ppc;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)(B * C), 1, 1);
+  cfg.blockDim = dim3(kRcThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)RcSmem::kBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, indexer_topk_rowcluster_kernel, tq, tk, p);
+  return e == cudaSuccess ? DS_OK : DS_ERR_CUDA;
+}
+
 static int indexer_check(const void* q, const void* kc, const float* w, int B, int H, int d, int S) {
   if (!q || !kc || !w || B <= 0 || H <= 0 || H > DS_INDEXER_MAX_HEADS || d != DS_INDEXER_DIM || S <= 0)
     return DS_ERR_ARG;
@@ -474,8 +642,12 @@ extern "C" int ds_indexer_topk(const void* q, const void* kcache, const float* w
   rc = device_state(&s);
   if (rc != DS_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (decode_fits(batch, heads, S, s))
-    return decode_enqueue(q, kcache, w, batch, heads, S, valid_len, k, out_idx, out_score, st, s);
+  if (!getenv("DS_INDEXER_UNFUSED")) {
+    if (decode_fits(batch, heads, S, s))
+      return decode_enqueue(q, kcache, w, batch, heads, S, valid_len, k, out_idx, out_score, st, s);
+    if (rowcluster_fits(batch, heads, S, s))
+      return rowcluster_enqueue(q, kcache, w, batch, heads, S, valid_len, k, out_idx, out_score, st, s);
+  }
   float* scores = static_cast<float*>(get_scratch(s, (size_t)batch * (size_t)S * sizeof(float)));
   if (!scores) return DS_ERR_NOMEM;
   rc = score_enqueue(q, kcache, w, batch, heads, S, valid_len, scores, st, s);

@@ -1,0 +1,652 @@
+// topk_stash_kernel.cuh -- row-wise top-k in one pass over the scores.
+//
+// What it computes: for each row, the k largest of the first L = valid_len
+// scores, ties to the lower position (DeepSelect hub page, use-case
+// paragraphs: top-k of a bfloat16 indexer score row, and of a float32 logit
+// row over a ~129K vocabulary; options sorted_index and return_value).
+//
+// How (B200 design, not the pages' design):
+//  * A row is handled by one CTA, or by a cluster of C = 2 or 4 CTAs that
+//    split it into contiguous slices when there are few rows.  Each CTA draws
+//    a strided sample of its slice and takes from it a key threshold t that,
+//    with a wide statistical margin, leaves at least min(k, slice) keys of the
+//    slice at or above it and not many more.  It then streams the slice once
+//    from HBM through a cp.async ring in shared memory and stashes every score
+//    whose key is >= t, with its position.
+//  * The k largest of a slice always contain that slice's share of the row's
+//    k largest, so a CTA only checks its own count: the stash must hold at
+//    least min(k, slice) keys and fit.  In a cluster every CTA then copies its
+//    stash into the leader CTA (distributed shared memory).
+//  * The leader selects the k largest of the stash by (key, lower position):
+//    one radix pass over the stash per digit (and, for keys equal to the k-th,
+//    over positions);
+//    every selected entry is written out with one warp-level atomic per
+//    visit, and sorted_index sorts the selection by position first.
+//  * A CTA whose stash came out short or too long (an unlucky sample, many
+//    equal keys) re-reads its slice from L2 and finds its exact k-th (key,
+//    position) with radix passes over the slice, then stashes exactly that
+//    many.
+#pragma once
+
+#include "ptx.cuh"
+#include "topk_kernel.cuh"
+
+namespace dstopk {
+
+constexpr int kTsThreads = 512;
+constexpr int kTsStages = 4;            // cp.async ring stages
+constexpr int kTsStageWords = 2048;     // 16-byte words per stage: a 128 KiB ring
+constexpr int kTsSample = 4096;         // sampled scores per CTA
+constexpr int kTsPosBits = 24;          // positions are below 2^24
+constexpr int kTsCap = 4096;            // stash entries per CTA (k <= 2048)
+constexpr int kTsMaxCluster = 4;
+
+struct TsParams {
+  const void* scores;
+  const int32_t* valid_len;
+  int32_t* out_idx;
+  void* out_val;
+  int batch, n, k;
+  int slice;         // elements per CTA, a multiple of 8
+  int return_value;
+  int sorted;
+};
+
+struct TsCtrl {
+  uint32_t cnt;             // this CTA: keys stashed (may run past the cap)
+  uint32_t out;             // leader: selected entries written
+  uint32_t bcast[4];
+  uint32_t ok[16];          // every CTA: each CTA's verdict
+  uint32_t tab[16];         // leader: each CTA's stash count
+  uint32_t wtot[32];        // scan scratch: warp totals
+  uint32_t wex[33];         // scan scratch: their exclusive prefixes, then the total
+  uint32_t part[32][kTsMaxCluster];  // per-warp partial counts
+  uint32_t above_of[kTsMaxCluster];
+};
+
+// Shared memory, in order: radix histogram u32[4096] (later the sorted
+// selection: positions u32[2048], raw scores u32[2048]) | control | this CTA's
+// stash (raw u32[cap], position u32[cap]) | cp.async ring of kTsStages stages.
+// The last ring stage holds the sample's histogram until the ring reaches it.
+// In a cluster the leader receives the stash of CTA c >= 1 in its ring (free
+// by then) at (c - 1) stash sizes.
+__host__ __device__ constexpr int ts_off_ctrl(int) { return 4096 * 4; }
+__host__ __device__ constexpr int ts_off_stash(int C) { return ts_off_ctrl(C) + 1024; }
+__host__ __device__ constexpr int ts_off_ring(int C) { return ts_off_stash(C) + kTsCap * 8; }
+__host__ __device__ constexpr int ts_ring_bytes() { return kTsStages * kTsStageWords * 16; }
+__host__ __device__ constexpr int ts_smem_bytes(int C) { return ts_off_ring(C) + ts_ring_bytes(); }
+static_assert(sizeof(TsCtrl) <= 1024, "control block");
+static_assert(ts_smem_bytes(kTsMaxCluster) <= 227 * 1024, "shared memory");
+static_assert((kTsMaxCluster - 1) * kTsCap * 8 <= ts_ring_bytes(), "received stashes fit the ring");
+
+// Exclusive block-wide scan of one value per thread (every thread calls it):
+// a shuffle scan in each warp, then warp 0 scans the warp totals.
+template <int NT>
+__device__ __forceinline__ uint32_t ts_block_scan(uint32_t v, TsCtrl* ctrl, uint32_t& total) {
+  static_assert(NT % 32 == 0 && NT / 32 <= 32, "one warp scans the warp totals");
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) ctrl->wtot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t x = lane < NW ? ctrl->wtot[lane] : 0u;
+    uint32_t y = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, y, o);
+      if (lane >= o) y += t;
+    }
+    if (lane < NW) ctrl->wex[lane] = y - x;
+    if (lane == 31) ctrl->wex[32] = y;
+  }
+  __syncthreads();
+  total = ctrl->wex[32];
+  return ctrl->wex[warp] + incl - v;
+}
+
+// In a histogram of nb bins find b with #(bins > b) < krem <= #(bins >= b);
+// `above` / `inbin` return the counts above and inside it.  Every thread calls
+// it and gets the result; a __syncthreads() must separate two calls.  Each
+// thread owns ceil(nb / NT) consecutive bins counted from the top.
+template <int NT>
+__device__ __forceinline__ uint32_t ts_find_bin(const uint32_t* h, int nb, uint32_t krem, TsCtrl* ctrl,
+                                                uint32_t& above, uint32_t& inbin) {
+  const int bpt = (nb + NT - 1) / NT;
+  const int r0 = (int)threadIdx.x * bpt;  // first rank (0 = the top bin)
+  const int r1 = min(nb, r0 + bpt);
+  uint32_t s = 0u;
+  if ((bpt & 3) == 0 && r1 - r0 == bpt) {
+    // bins nb-r1 .. nb-1-r0 are 16-byte aligned groups of four
+    for (int r = r0; r < r1; r += 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(h + nb - 4 - r);
+      s += v.x + v.y + v.z + v.w;
+    }
+  } else {
+    for (int r = r0; r < r1; ++r) s += h[nb - 1 - r];
+  }
+  if (threadIdx.x == 0) {
+    ctrl->bcast[0] = 0u;
+    ctrl->bcast[1] = 0u;
+    ctrl->bcast[2] = 0u;
+  }
+  uint32_t total;
+  const uint32_t excl = ts_block_scan<NT>(s, ctrl, total);
+  if (excl < krem && krem <= excl + s) {
+    uint32_t acc = excl;
+    for (int r = r0; r < r1; ++r) {
+      const uint32_t c = h[nb - 1 - r];
+      if (acc + c >= krem) {
+        ctrl->bcast[0] = (uint32_t)(nb - 1 - r);
+        ctrl->bcast[1] = acc;
+        ctrl->bcast[2] = c;
+        break;
+      }
+      acc += c;
+    }
+  }
+  __syncthreads();
+  above = ctrl->bcast[1];
+  inbin = ctrl->bcast[2];
+  return min(ctrl->bcast[0], (uint32_t)(nb - 1));
+}
+
+// Radix digits of the key, most significant first: 12 / 11 / 9 (float32) or
+// 12 / 4 (bfloat16) bits.
+template <class K>
+struct TsDigits;
+template <>
+struct TsDigits<F32Keys> {
+  static constexpr int kCount = 3;
+  __device__ __forceinline__ static int width(int i) { return i == 0 ? 12 : (i == 1 ? 11 : 9); }
+};
+template <>
+struct TsDigits<BF16Keys> {
+  static constexpr int kCount = 2;
+  __device__ __forceinline__ static int width(int i) { return i == 0 ? 12 : 4; }
+};
+
+// Where an exact selection of the kth largest (key, then lower position)
+// cuts: an element is taken when the top bits of its key (key >> kshift)
+// exceed kprefix, or equal it and its position is <= pcut.
+struct TsCut {
+  uint32_t kprefix;
+  int kshift;
+  uint32_t pcut;
+};
+
+__device__ __forceinline__ uint32_t ts_top(uint32_t key, int shift) { return shift >= 32 ? 0u : key >> shift; }
+
+__device__ __forceinline__ bool ts_taken(const TsCut& c, uint32_t key, uint32_t pos) {
+  const uint32_t top = ts_top(key, c.kshift);
+  return top > c.kprefix || (top == c.kprefix && pos <= c.pcut);
+}
+
+// Exact radix select of the kth largest (key, lower position) among the
+// elements that visit(f) hands to f(key, position) (at least kth of them,
+// kth >= 1; positions below 2^24 and distinct).  Radix passes on the key;
+// only if ties at the kth key remain, two 12-bit passes on the complemented
+// positions of the tied elements.  Every thread of the block calls it.
+// When first_ready is set, hist already holds the histogram of the first
+// digit (the top 12 key bits) of those elements.  With start_pass = 1 every
+// visited element has first digit prefix0 and inbin0 elements are visited.
+template <class K, int NT, class Visit>
+__device__ __forceinline__ TsCut ts_select(Visit&& visit, int kth, uint32_t* hist, TsCtrl* ctrl,
+                                           bool first_ready = false, int start_pass = 0, uint32_t prefix0 = 0u,
+                                           uint32_t inbin0 = 0u) {
+  uint32_t prefix = 0;
+  int shift = K::kBits;
+  int krem = kth;
+  if (start_pass == 1) {
+    prefix = prefix0;
+    shift = K::kBits - TsDigits<K>::width(0);
+    if (inbin0 == (uint32_t)kth) return TsCut{prefix, shift, 0xFFFFFFFFu};
+  }
+  for (int pass = start_pass; pass < TsDigits<K>::kCount; ++pass) {
+    const int wd = TsDigits<K>::width(pass);
+    const int sh = shift - wd;
+    const uint32_t mask = (1u << wd) - 1u;
+    if (pass > 0 || !first_ready) {
+      for (int i = threadIdx.x; i <= (int)mask; i += NT) hist[i] = 0u;
+      __syncthreads();
+      const uint32_t pf = prefix;
+      const int sf = shift;
+      visit([&](uint32_t key, uint32_t) {
+        if (ts_top(key, sf) == pf) atomicAdd(hist + ((key >> sh) & mask), 1u);
+      });
+      __syncthreads();
+    }
+    uint32_t above, inbin;
+    const uint32_t b = ts_find_bin<NT>(hist, (int)mask + 1, (uint32_t)krem, ctrl, above, inbin);
+    krem -= (int)above;
+    prefix = (prefix << wd) | b;
+    shift = sh;
+    if (inbin == (uint32_t)krem) return TsCut{prefix, shift, 0xFFFFFFFFu};  // the whole bin is taken
+  }
+  // prefix is the kth key; krem of its ties are taken, the lowest positions first
+  const uint32_t tkey = prefix;
+  uint32_t pp = 0;
+  int ps = kTsPosBits;
+  for (int pass = 0; pass < 2; ++pass) {
+    const int sh = ps - 12;
+    for (int i = threadIdx.x; i < 4096; i += NT) hist[i] = 0u;
+    __syncthreads();
+    const uint32_t pf = pp;
+    const int sf = ps;
+    visit([&](uint32_t key, uint32_t pos) {
+      const uint32_t cp = ((1u << kTsPosBits) - 1u) - pos;
+      if (key == tkey && (cp >> sf) == pf) atomicAdd(hist + ((cp >> sh) & 4095u), 1u);
+    });
+    __syncthreads();
+    uint32_t above, inbin;
+    const uint32_t b = ts_find_bin<NT>(hist, 4096, (uint32_t)krem, ctrl, above, inbin);
+    krem -= (int)above;
+    pp = (pp << 12) | b;
+    ps = sh;
+    if (inbin == (uint32_t)krem) break;
+  }
+  // taken ties: complemented position >= pp << ps
+  return TsCut{tkey, 0, ((1u << kTsPosBits) - 1u) - (pp << ps)};
+}
+
+// Hands out n consecutive slots of *counter to each lane of a warp (all 32
+// lanes call it); returns this lane's first slot.
+__device__ __forceinline__ uint32_t ts_warp_alloc(uint32_t n, uint32_t* counter) {
+  const int lane = threadIdx.x & 31;
+  uint32_t incl = n;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+  uint32_t base = 0;
+  if (total != 0u) {
+    if (lane == 0) base = atomicAdd(counter, total);
+    base = __shfl_sync(0xFFFFFFFFu, base, 0);
+  }
+  return base + incl - n;
+}
+
+
+
+// Block-wide sums of C <= kTsMaxCluster values per thread (every thread calls
+// it); the sums land in out[0 .. C).
+template <int NT>
+__device__ __forceinline__ void ts_block_sums(const uint32_t (&v)[kTsMaxCluster], int C, TsCtrl* ctrl,
+                                              uint32_t* out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int c = 0; c < kTsMaxCluster; ++c) {
+    uint32_t x = v[c];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
+    if (lane == 0) ctrl->part[warp][c] = x;
+  }
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int c = 0; c < kTsMaxCluster; ++c) {
+      uint32_t x = lane < NT / 32 ? ctrl->part[lane][c] : 0u;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
+      if (lane == 0 && c < C) out[c] = x;
+    }
+  }
+  __syncthreads();
+}
+
+template <class K, int NT>
+__global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  using Raw = typename K::Raw;
+  constexpr int kShift0 = K::kBits - 12;
+  constexpr int stage_words = kTsStageWords;
+  constexpr int V = stage_words / NT;  // words per thread per stage
+  static_assert(V * NT == stage_words && V * K::kVec <= 64, "ring stage");
+
+  const int tid = threadIdx.x;
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t csize = cluster_nctarank();
+  const int C = (int)csize;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem);  // radix histogram
+  TsCtrl* ctrl = reinterpret_cast<TsCtrl*>(smem + ts_off_ctrl(C));
+  uint32_t* st_raw = reinterpret_cast<uint32_t*>(smem + ts_off_stash(C));
+  uint32_t* st_pos = st_raw + kTsCap;
+  uint8_t* ring = smem + ts_off_ring(C);
+  uint32_t* shist = reinterpret_cast<uint32_t*>(ring + (size_t)(kTsStages - 1) * stage_words * 16);
+
+  const int row = (int)(blockIdx.x / csize);
+  int L = p.n;
+  if (p.valid_len) {
+    const int v = p.valid_len[row];
+    L = v < 0 ? 0 : (v > p.n ? p.n : v);
+  }
+  const int kk = min(p.k, L);
+  int32_t* out_idx = p.out_idx + (size_t)row * p.k;
+  Raw* out_val = p.return_value ? reinterpret_cast<Raw*>(p.out_val) + (size_t)row * p.k : nullptr;
+  if (crank == 0) {
+    for (int j = kk + tid; j < p.k; j += NT) {
+      out_idx[j] = -1;
+      if (out_val) out_val[j] = (Raw)K::kNegInf;
+    }
+  }
+  if (kk == 0) return;  // uniform across the cluster
+
+  const int i0 = (int)crank * p.slice;
+  const int m = max(0, min(p.slice, L - i0));  // eligible scores of this slice
+  const int need = min(kk, m);                 // the stash must hold at least this many
+  const Raw* grow = reinterpret_cast<const Raw*>(p.scores) + (size_t)row * p.n;
+
+  // the slice as full 16-byte words plus fewer than 2 * kVec loose elements
+  const uintptr_t rbase = reinterpret_cast<uintptr_t>(grow);
+  const uintptr_t a0 = rbase + (uintptr_t)i0 * K::kBytes;
+  const uintptr_t a1 = a0 + (uintptr_t)m * K::kBytes;
+  const uintptr_t f0 = (a0 + 15u) & ~uintptr_t(15);
+  const uintptr_t f1 = a1 & ~uintptr_t(15);
+  const int nfull = (m > 0 && f1 > f0) ? (int)((f1 - f0) >> 4) : 0;
+  const uint4* wp = reinterpret_cast<const uint4*>(f0);
+  const int e_f0 = (int)((f0 - rbase) / K::kBytes);
+  const int head = m <= 0 ? 0 : (nfull > 0 ? (int)((f0 - a0) / K::kBytes) : m);
+  const int tail_start = nfull > 0 ? (int)((f1 - rbase) / K::kBytes) : i0 + m;
+  const int tail = m <= 0 ? 0 : i0 + m - tail_start;
+  int pe = -1;  // this thread's loose element, if any
+  if (tid < head) pe = i0 + tid;
+  else if (nfull > 0 && tid >= 32 && tid - 32 < tail) pe = tail_start + tid - 32;
+
+  if (tid == 0) {
+    ctrl->cnt = 0u;
+    ctrl->out = 0u;
+  }
+
+  // ---- a strided sample of the full words (64 evenly spaced runs of run_w
+  // words) when the slice does not fit the stash whole
+  constexpr int SW = kTsSample / K::kVec;
+  constexpr int SPT = (SW + NT - 1) / NT;
+  constexpr int kRuns = 64;
+  const bool sampled = m > kTsCap;
+  const int run_w = sampled ? min(nfull, SW) / kRuns : 0;  // >= 7: a sampled slice has > 4096 scores
+  const int sw = kRuns * run_w;                            // sampled words, <= nfull
+  uint4 s[SPT];
+#pragma unroll
+  for (int j = 0; j < SPT; ++j) {
+    const int idx = tid + j * NT;
+    if (idx < sw) {
+      const int ru = idx / run_w, o = idx - ru * run_w;
+      s[j] = __ldg(wp + (int)(((long long)ru * (nfull - run_w)) / (kRuns - 1)) + o);
+    }
+  }
+  uint32_t praw = 0;
+  if (pe >= 0) praw = (uint32_t)grow[pe];
+
+  // ---- the cp.async ring: a thread copies V words per stage and later
+  // processes exactly those words, so the ring needs no block barrier
+  const int nst = (nfull + stage_words - 1) / stage_words;
+  auto issue = [&](int st) {
+    if (st < nst) {
+      const int slot = st % kTsStages;
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        const int w = st * stage_words + v * NT + tid;
+        if (w < nfull) {
+          const uint32_t dst = smem_u32(ring + ((size_t)slot * stage_words + v * NT + tid) * 16);
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(wp + w) : "memory");
+        }
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  // ---- threshold: the sample's key of rank rk, which leaves an expected
+  // need + 4 standard deviations + 8 keys of the slice above it
+  uint32_t t = 0u;
+  if (sampled) {
+    for (int i = tid; i < 4096; i += NT) shist[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < SPT; ++j) {
+      if (tid + j * NT < sw) {
+#pragma unroll
+        for (int e = 0; e < K::kVec; ++e) atomicAdd(shist + (K::key(K::slot(s[j], e)) >> kShift0), 1u);
+      }
+    }
+    for (int st = 0; st < kTsStages - 1; ++st) issue(st);  // the sample has landed: start the stream
+    __syncthreads();
+    const int ns = sw * K::kVec;
+    const float lam = (float)need * (float)ns / (float)m;
+    const int rk = min(ns, (int)ceilf(lam + 4.0f * sqrtf(lam) + 8.0f));
+    uint32_t above, inbin;
+    const uint32_t b1 = ts_find_bin<NT>(shist, 4096, (uint32_t)rk, ctrl, above, inbin);
+    constexpr int W2 = kShift0 >= 11 ? 11 : kShift0;
+    constexpr int SH2 = kShift0 - W2;
+    for (int i = tid; i < (1 << W2); i += NT) shist[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < SPT; ++j) {
+      if (tid + j * NT < sw) {
+#pragma unroll
+        for (int e = 0; e < K::kVec; ++e) {
+          const uint32_t kv = K::key(K::slot(s[j], e));
+          if ((kv >> kShift0) == b1) atomicAdd(shist + ((kv >> SH2) & ((1u << W2) - 1u)), 1u);
+        }
+      }
+    }
+    __syncthreads();
+    uint32_t a2, i2;
+    const uint32_t b2 = ts_find_bin<NT>(shist, 1 << W2, (uint32_t)(rk - (int)above), ctrl, a2, i2);
+    t = ((b1 << W2) | b2) << SH2;
+  } else {
+    for (int st = 0; st < kTsStages - 1; ++st) issue(st);
+    __syncthreads();  // the zeroed histogram and counters
+  }
+
+  // ---- one pass: every key >= t is stashed with its position and its first
+  // digit counted; a warp takes its stash slots with one atomic per stage
+  for (int st = 0; st < nst; ++st) {
+    issue(st + kTsStages - 1);
+    asm volatile("cp.async.wait_group %0;" ::"n"(kTsStages - 1) : "memory");
+    const int slot = st % kTsStages;
+    uint4 x[V];
+    unsigned long long hits = 0ull;
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const int w = st * stage_words + v * NT + tid;
+      x[v] = make_uint4(0u, 0u, 0u, 0u);
+      if (w < nfull) {
+        x[v] = *reinterpret_cast<const uint4*>(ring + ((size_t)slot * stage_words + v * NT + tid) * 16);
+#pragma unroll
+        for (int j = 0; j < K::kVec; ++j)
+          hits |= (unsigned long long)(K::key(K::slot(x[v], j)) >= t) << (v * K::kVec + j);
+      }
+    }
+    uint32_t pos = ts_warp_alloc((uint32_t)__popcll(hits), &ctrl->cnt);
+    if (hits) {
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        const int e0 = e_f0 + (st * stage_words + v * NT + tid) * K::kVec;
+#pragma unroll
+        for (int j = 0; j < K::kVec; ++j) {
+          if ((hits >> (v * K::kVec + j)) & 1ull) {
+            if (pos < (uint32_t)kTsCap) {
+              st_raw[pos] = K::slot(x[v], j);
+              st_pos[pos] = (uint32_t)(e0 + j);
+            }
+            ++pos;
+          }
+        }
+      }
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  if (pe >= 0) {
+    const uint32_t key = K::key(praw);
+    if (key >= t) {
+      const uint32_t slot = atomicAdd(&ctrl->cnt, 1u);
+      if (slot < (uint32_t)kTsCap) {
+        st_raw[slot] = praw;
+        st_pos[slot] = (uint32_t)pe;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- in a cluster, every stash and histogram goes to the leader: stash c
+  // into the leader's ring (free once every CTA has streamed) at (c - 1) stash
+  // sizes, histogram c into its slot c
+  auto region = [&](int c) -> uint32_t* {
+    return c == 0 ? st_raw : reinterpret_cast<uint32_t*>(ring + (size_t)(c - 1) * kTsCap * 8);
+  };
+  auto ship = [&](uint32_t n) {
+    const uint32_t nv = (n + 3u) >> 2;
+    const uint32_t dst = dsmem_map(smem_u32(region((int)crank)), 0);
+    for (uint32_t v = tid; v < 2u * nv; v += NT) {
+      const bool israw = v < nv;
+      const uint32_t o = 16u * (israw ? v : v - nv);
+      const uint4 x = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(israw ? st_raw : st_pos) + o);
+      asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst + (israw ? 0u : 4u * kTsCap) + o),
+                   "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w)
+                   : "memory");
+    }
+    if (tid == 0) dsmem_st_u32(dsmem_map(smem_u32(&ctrl->tab[crank]), 0), n);
+  };
+
+  uint32_t cnt = ctrl->cnt;
+  const bool ok = cnt >= (uint32_t)need && cnt <= (uint32_t)kTsCap;
+  bool all_ok = ok;
+  if (C > 1) {
+    cluster_sync();  // every CTA has streamed: the leader's ring is free
+    if (ok && crank != 0) ship(cnt);
+    if (tid < C) dsmem_st_u32(dsmem_map(smem_u32(&ctrl->ok[crank]), (uint32_t)tid), ok ? 1u : 0u);
+    cluster_sync();
+    for (int c = 0; c < C; ++c) all_ok &= ctrl->ok[c] != 0u;
+  }
+  if (tid == 0 && crank == 0) ctrl->tab[0] = cnt;
+
+  if (!all_ok) {
+    // ---- exact fallback (uniform decision; only CTAs with a bad stash work):
+    // radix passes over the slice (re-read from L2) find its need-th largest
+    // (key, lower position); then exactly its need largest are stashed
+    if (!ok) {
+      auto visit_slice = [&](auto&& f) {
+        stream_slice<K, NT, 4>(
+            grow, i0, m,
+            [&](int e0, const uint4& v) {
+#pragma unroll
+              for (int j = 0; j < K::kVec; ++j) f(K::key(K::slot(v, j)), (uint32_t)(e0 + j));
+            },
+            [&](int e, uint32_t raw) { f(K::key(raw), (uint32_t)e); });
+      };
+      const TsCut cut = ts_select<K, NT>(visit_slice, need, hist, ctrl);
+      if (tid == 0) ctrl->cnt = 0u;
+      __syncthreads();
+      auto take = [&](uint32_t raw, int e) {
+        const uint32_t key = K::key(raw);
+        if (ts_taken(cut, key, (uint32_t)e)) {
+          const uint32_t slot = atomicAdd(&ctrl->cnt, 1u);
+          if (slot < (uint32_t)kTsCap) {
+            st_raw[slot] = raw;
+            st_pos[slot] = (uint32_t)e;
+          }
+        }
+      };
+      stream_slice<K, NT, 4>(
+          grow, i0, m,
+          [&](int e0, const uint4& v) {
+#pragma unroll
+            for (int j = 0; j < K::kVec; ++j) take(K::slot(v, j), e0 + j);
+          },
+          [&](int e, uint32_t raw) { take(raw, e); });
+      __syncthreads();
+      cnt = ctrl->cnt;  // == need
+      if (crank != 0) ship(cnt);
+      else if (tid == 0) ctrl->tab[0] = cnt;
+    }
+    if (C > 1) cluster_sync();
+    else __syncthreads();
+  }
+  if (crank != 0) return;
+
+  // ---- the leader: the kk largest of the (merged) stash
+  __syncthreads();
+  auto visit_stash = [&](auto&& f) {
+    for (int c = 0; c < C; ++c) {
+      const int nc = min((int)ctrl->tab[c], kTsCap);
+      const uint32_t* rr = region(c);
+      const uint32_t* rp = rr + kTsCap;
+      int i = tid;
+      for (; i + NT < nc; i += 2 * NT) {
+        const uint32_t a0 = rr[i], a1 = rr[i + NT], q0 = rp[i], q1 = rp[i + NT];
+        f(K::key(a0), q0);
+        f(K::key(a1), q1);
+      }
+      if (i < nc) f(K::key(rr[i]), rp[i]);
+    }
+  };
+  const TsCut cut = ts_select<K, NT>(visit_stash, kk, hist, ctrl);
+  // every selected entry (exactly kk): one warp-level slot allocation per
+  // visit; with sorted_index gathered in shared memory first
+  uint32_t* sel_pos = hist;
+  uint32_t* sel_raw = hist + 2048;
+  const bool sorted = p.sorted != 0;
+  for (int c = 0; c < C; ++c) {
+    const int nc = min((int)ctrl->tab[c], kTsCap);
+    const uint32_t* rr = region(c);
+    const uint32_t* rp = rr + kTsCap;
+    for (int base = 0; base < nc; base += NT) {
+      const int i = base + tid;
+      uint32_t raw = 0u, pos = 0u;
+      bool take = false;
+      if (i < nc) {
+        raw = rr[i];
+        pos = rp[i];
+        take = ts_taken(cut, K::key(raw), pos);
+      }
+      const uint32_t slot = ts_warp_alloc(take ? 1u : 0u, &ctrl->out);
+      if (take && slot < (uint32_t)kk) {
+        if (sorted) {
+          sel_pos[slot] = pos;
+          sel_raw[slot] = raw;
+        } else {
+          out_idx[slot] = (int32_t)pos;
+          if (out_val) out_val[slot] = (Raw)raw;
+        }
+      }
+    }
+  }
+  if (!sorted) return;
+  __syncthreads();
+  // ascending positions: bitonic sort of (position, score) pairs
+  int np = 1;
+  while (np < kk) np <<= 1;
+  for (int i = kk + tid; i < np; i += NT) sel_pos[i] = 0xFFFFFFFFu;
+  __syncthreads();
+  for (int len = 2; len <= np; len <<= 1) {
+    for (int st = len >> 1; st > 0; st >>= 1) {
+      for (int i = tid; i < np; i += NT) {
+        const int j = i ^ st;
+        if (j > i) {
+          const uint32_t a = sel_pos[i], b = sel_pos[j];
+          if ((a > b) == ((i & len) == 0)) {
+            sel_pos[i] = b;
+            sel_pos[j] = a;
+            const uint32_t x = sel_raw[i];
+            sel_raw[i] = sel_raw[j];
+            sel_raw[j] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int j = tid; j < kk; j += NT) {
+    out_idx[j] = (int32_t)sel_pos[j];
+    if (out_val) out_val[j] = (Raw)sel_raw[j];
+  }
+}
+
+}  // namespace dstopk

@@ -228,3 +228,104 @@ def test_fused_decode_graph_replay_with_odd_call_count(cuda_device, grid_fused):
         assert ds.ds_get_device_status() == ds.DS_OK
         for o in outs:
             check_selection(q, kc, w, vl, 512, o.cpu().numpy(), None)
+
+
+# ---------------------------------------------------------------- row-per-cluster path
+
+@pytest.fixture
+def rowcluster(monkeypatch):
+    # one cluster per row, whatever the batch (the default takes it for small batches)
+    monkeypatch.setenv("DS_INDEXER_ROWCLUSTER", "1")
+
+
+def test_rowcluster_matches_unfused_path(cuda_device, rowcluster, monkeypatch):
+    # both paths compute the float32 scores in the same order (tensor-core dot
+    # products, then the weighted head sum from head 0 up), so they select the
+    # same positions and return the same scores
+    q, kc, w, vl = inputs.decode(seed=37)
+    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
+    got, gs = ds.ds_indexer_topk(qd, kd, wd, 1024, valid_len=vd, return_score=True)
+    torch.cuda.synchronize()
+    monkeypatch.setenv("DS_INDEXER_UNFUSED", "1")
+    ref, rs = ds.ds_indexer_topk(qd, kd, wd, 1024, valid_len=vd, return_score=True)
+    torch.cuda.synchronize()
+    assert ds.ds_get_device_status() == ds.DS_OK
+    g, r = got.cpu().numpy(), ref.cpu().numpy()
+    for t in range(q.shape[0]):
+        assert np.array_equal(np.sort(g[t]), np.sort(r[t])), f"row {t}"
+        og, orr = np.argsort(g[t]), np.argsort(r[t])
+        assert np.array_equal(gs.cpu().numpy()[t][og], rs.cpu().numpy()[t][orr])
+
+
+@pytest.mark.parametrize("B,H,S,k", [(1, 64, 32768, 2048), (16, 64, 32768, 1024), (5, 64, 7000, 512),
+                                     (8, 64, 128, 64), (2, 64, 129, 2048), (3, 40, 20000, 100),
+                                     (4, 64, 300, 1), (20, 64, 5000, 256)])
+def test_rowcluster_shapes(cuda_device, rowcluster, B, H, S, k):
+    q, kc, w = inputs.indexer_factors(seed=B * 5 + S + H, batch=B, n=S, heads=H)
+    g = np.random.default_rng(S + B)
+    vl = g.integers(-3, S + 5, size=B).astype(np.int32)
+    vl[0] = S
+    if B > 1:
+        vl[1] = 0
+    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
+    idx, score = ds.ds_indexer_topk(qd, kd, wd, k, valid_len=vd, return_score=True)
+    torch.cuda.synchronize()
+    assert ds.ds_get_device_status() == ds.DS_OK
+    check_selection(q, kc, w, vl, k, idx.cpu().numpy(), score.cpu().numpy())
+
+
+@pytest.mark.parametrize("B,H,S,k", [(8, 64, 32768, 2048), (3, 64, 5000, 1000), (2, 24, 777, 700)])
+def test_rowcluster_exact_arithmetic(cuda_device, rowcluster, B, H, S, k):
+    # small-integer inputs: exact float32 scores with many equal values, so the
+    # index sets must match the oracle's exactly, ties to the lower position
+    q, kc, w = exact_inputs(B * 13 + S, B, H, S)
+    qd, kd, wd, _ = dev_inputs(q, kc, w, None)
+    idx, score = ds.ds_indexer_topk(qd, kd, wd, k, return_score=True)
+    torch.cuda.synchronize()
+    assert ds.ds_get_device_status() == ds.DS_OK
+    ref_idx, ref_scores = oracle.indexer_topk(q, kc, w, k)
+    idx, score = idx.cpu().numpy(), score.cpu().numpy()
+    for t in range(B):
+        m = int((ref_idx[t] >= 0).sum())
+        assert np.array_equal(np.sort(idx[t, :m]), np.sort(ref_idx[t, :m])), f"row {t}"
+        assert np.array_equal(score[t, :m].astype(np.float64), ref_scores[t, idx[t, :m]])
+
+
+@pytest.mark.parametrize("S,L", [(32768, 32768), (20000, 12000), (4096, 4000)])
+def test_rowcluster_all_scores_equal(cuda_device, rowcluster, S, L):
+    # zero weights: every score is 0, the whole row sits in one radix bin (past
+    # the leader's list capacity for the longest rows) and the k lowest
+    # positions must be returned
+    q, kc, w = inputs.indexer_factors(seed=S, batch=2, n=S, heads=64)
+    w = np.zeros_like(w)
+    vl = np.array([L, L // 3], dtype=np.int32)
+    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
+    idx, score = ds.ds_indexer_topk(qd, kd, wd, 2048, valid_len=vd, return_score=True)
+    torch.cuda.synchronize()
+    assert ds.ds_get_device_status() == ds.DS_OK
+    idx = idx.cpu().numpy()
+    for t in range(2):
+        m = min(2048, int(vl[t]))
+        assert np.array_equal(np.sort(idx[t, :m]), np.arange(m)), f"row {t}"
+        assert np.all(idx[t, m:] == -1)
+    assert np.all(score.cpu().numpy()[:, :min(2048, L // 3)] == 0.0)
+
+
+def test_rowcluster_graph_replay(cuda_device, rowcluster):
+    q, kc, w, vl = inputs.decode(seed=43, S=8192, vl_lo=1000, vl_hi=8192)
+    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
+    outs = [torch.empty((8, 512), dtype=torch.int32, device="cuda") for _ in range(3)]
+    ds.ds_indexer_topk(qd, kd, wd, 512, valid_len=vd, out_idx=outs[0])
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for o in outs:
+            ds.ds_indexer_topk(qd, kd, wd, 512, valid_len=vd, out_idx=o)
+    for _ in range(2):
+        for o in outs:
+            o.fill_(-7)
+        gr.replay()
+        torch.cuda.synchronize()
+        assert ds.ds_get_device_status() == ds.DS_OK
+        for o in outs:
+            check_selection(q, kc, w, vl, 512, o.cpu().numpy(), None)
