@@ -33,7 +33,7 @@
 
 namespace dstopk {
 
-constexpr int kTsThreads = 512;
+constexpr int kTsThreads = 1024;
 constexpr int kTsStages = 4;            // cp.async ring stages
 constexpr int kTsStageWords = 2048;     // 16-byte words per stage: a 128 KiB ring
 constexpr int kTsSample = 4096;         // sampled scores per CTA
