@@ -41,6 +41,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 1024 * 1024
 
 SAMPLING = dict(batch=64, n=129280, ks=(1024, 64))
+# ds_topk runs the one-pass stash kernel for >= 32 rows (the cluster kernel below)
+TOPK_KERNEL = "topk_stash_kernel<F32Keys, 1024>"
 DECODE = dict(batch=8, heads=64, d=128, S=32768, k=1024)
 
 
@@ -346,13 +348,15 @@ def run_ours(args):
     h2d = xb
     d2h = B * (k1 + k2) * 8
 
+    # DRAM bytes per launch of the dominant kernel from one ncu capture; null
+    # once the kernel's source has changed since that capture
     traffic = None
     prof = os.path.join(ROOT, "profiles", "topk_traffic.json")
     try:
         import hashlib
         with open(prof) as f:
             pj = json.load(f)
-        src = open(os.path.join(ROOT, "sparse_attention_top_ds_b200", "csrc", "topk_kernel.cuh"), "rb").read()
+        src = open(os.path.join(ROOT, "sparse_attention_top_ds_b200", "csrc", pj["kernel_source"]), "rb").read()
         if pj.get("kernel_source_sha256") == hashlib.sha256(src).hexdigest():
             traffic = pj.get("dram_bytes_per_launch")
     except Exception:
@@ -384,7 +388,7 @@ def run_ours(args):
             "decode_frac_of_roofline": round(dec_roof_us / (t_dec * 1e3), 3),
             "roofline": {"bound": "hbm", "achieved": round(per_launch_gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
                          "frac": round(per_launch_gbs / hbm_gbs, 4), "traffic": traffic,
-                         "kernel": "topk_cluster_kernel<F32Keys>", "peak_source": peak_src},
+                         "kernel": TOPK_KERNEL, "peak_source": peak_src},
             "e2e": {"value": round(e2e_gbs, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": 4 * args.steps,
             "clocks": clocks,
