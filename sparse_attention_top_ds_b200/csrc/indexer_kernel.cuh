@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
   const int tile_lo = part * p.tiles_per_cta;
   const int tile_hi = min(ntiles, tile_lo + p.tiles_per_cta);
 
+  pdl_wait();
   // largest valid length in the group: tiles at or past it are not computed
   int maxvl = 0;
   for (int t = 0; t < NT; ++t) {
@@ -263,6 +264,9 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+  // the next kernel (the top-k over these rows) may launch only now: launched
+  // earlier its CTAs would crowd onto the few SMs this grid leaves free
+  pdl_launch_dependents();
 }
 
 }  // namespace dstopk

@@ -55,6 +55,18 @@ static bool topk_cluster16_ok();
 static int rowcluster_active(int C);
 static int g_max_cluster = 8;  // largest cluster the top-k launch may use
 
+// Launch attribute: the kernel may start while the previous kernel on the
+// stream finishes (every kernel launched with it waits, with griddepcontrol,
+// before it touches global memory).  DS_NO_PDL=1 turns it off (comparisons).
+static bool pdl_on() {
+  static const bool on = getenv("DS_NO_PDL") == nullptr;
+  return on;
+}
+static void set_pdl(cudaLaunchAttribute& a) {
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+}
+
 // Set-up once per device, with that device current: capability check, the
 // status word's address, and the kernels' shared-memory limits.
 static int device_state(DeviceState** out) {
@@ -172,13 +184,14 @@ static cudaError_t launch_topk(const TopkParams& p, int C, cudaStream_t st) {
   cfg.blockDim = dim3(NT, 1, 1);
   cfg.dynamicSmemBytes = (size_t)kTopkSmemBytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  set_pdl(attr[1]);
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_on() ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, topk_cluster_kernel<K, NT>, p);
 }
 
@@ -216,13 +229,14 @@ static int topk_stash_enqueue(const void* scores, int batch, int n, int k, int d
   cfg.blockDim = dim3(kTsThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)ts_smem_bytes(C);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  set_pdl(attr[1]);
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_on() ? 2 : 1;
   int nt = kTsThreads;
   const char* fnt = getenv("DS_TOPK_NT");  // tuning sweeps only
   if (fnt && (atoi(fnt) == 256 || atoi(fnt) == 512 || atoi(fnt) == 1024)) nt = atoi(fnt);
@@ -387,8 +401,18 @@ static int launch_score(const void* q, const void* kc, const float* w, int B, in
   p.S = S;
   p.tiles_per_cta = (int)tpc;
   p.ctas_per_group = cpg;
-  indexer_score_kernel<NT, HP, ST><<<groups * cpg, Cfg::kThreads, Cfg::kSmemBytes, st>>>(tq, tk, p);
-  return cudaGetLastError() == cudaSuccess ? DS_OK : DS_ERR_CUDA;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)(groups * cpg), 1, 1);
+  cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)Cfg::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  set_pdl(attr[0]);
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_on() ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, indexer_score_kernel<NT, HP, ST>, tq, tk, p);
+  return e == cudaSuccess ? DS_OK : DS_ERR_CUDA;
 }
 
 static int score_enqueue(const void* q, const void* kc, const float* w, int B, int H, int S, const int32_t* vl,

@@ -165,3 +165,19 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
 }
 
 }  // namespace dstopk
+
+namespace dstopk {
+
+// ------------------------------------------------------------------ programmatic dependent launch
+//
+// Kernels launched with cudaLaunchAttributeProgrammaticStreamSerialization may
+// start while the previous kernel on the stream is finishing.  Each such kernel
+// waits for the previous kernel's completion (and its memory) before it touches
+// global memory, and lets the next kernel start launching once all of its own
+// CTAs are resident.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace dstopk

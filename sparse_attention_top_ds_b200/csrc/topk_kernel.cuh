@@ -286,6 +286,8 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_cluster_kernel(const TopkP
   const uint32_t crank = cluster_ctarank();
   const uint32_t csize = cluster_nctarank();
   const int row = blockIdx.x / csize;
+  pdl_wait();
+  pdl_launch_dependents();
 
   int L = p.n;
   if (p.valid_len) {

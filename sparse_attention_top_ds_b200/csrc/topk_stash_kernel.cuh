@@ -322,6 +322,8 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   uint32_t* shist = reinterpret_cast<uint32_t*>(ring + (size_t)(kTsStages - 1) * stage_words * 16);
 
   const int row = (int)(blockIdx.x / csize);
+  pdl_wait();
+  pdl_launch_dependents();
   int L = p.n;
   if (p.valid_len) {
     const int v = p.valid_len[row];
