@@ -44,6 +44,7 @@ SAMPLING = dict(batch=64, n=129280, ks=(1024, 64))
 # ds_topk runs the one-pass stash kernel for >= 32 rows (the cluster kernel below)
 TOPK_KERNEL = "topk_stash_kernel<F32Keys, 1024>"
 DECODE = dict(batch=8, heads=64, d=128, S=32768, k=1024)
+PREFILL = dict(k=2048)
 
 
 def load_peaks():
@@ -350,6 +351,45 @@ def run_ours(args):
 
     # DRAM bytes per launch of the dominant kernel from one ncu capture; null
     # once the kernel's source has changed since that capture
+    # ---- prefill, reported beside the headline: 4096 query rows x 64 heads
+    # against 32768 keys, causal valid_len, k = 2048 (indexer + top-k per call,
+    # and the scorer alone for its tensor-pipe fraction)
+    pq, pkc, pw, pvl = inputs.prefill(seed=inputs.SEED_PREFILL + rank)
+    pq_d = torch.from_numpy(pq.view(np.int16)).view(torch.bfloat16).to(dev)
+    pkc_d = torch.from_numpy(pkc.view(np.int16)).view(torch.bfloat16).to(dev)
+    pw_d = torch.from_numpy(pw).to(dev)
+    pvl_d = torch.from_numpy(pvl).to(dev)
+    T = pq.shape[0]
+    pidx = torch.empty((T, PREFILL["k"]), dtype=torch.int32, device=dev)
+    pscore = torch.empty((T, pkc.shape[0]), dtype=torch.float32, device=dev)
+
+    def time_calls(fn, calls=3):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(calls):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) / calls
+
+    pre_ms = time_calls(lambda: ds.ds_indexer_topk(pq_d, pkc_d, pw_d, PREFILL["k"], valid_len=pvl_d, out_idx=pidx))
+    pre_score_ms = time_calls(lambda: ds.ds_indexer_score(pq_d, pkc_d, pw_d, valid_len=pvl_d, out=pscore))
+    pre_ms, pre_score_ms = max_over_ranks([pre_ms, pre_score_ms], dev)
+    pre_flops = 2.0 * pq.shape[1] * pq.shape[2] * float(np.sum(pvl.astype(np.int64)))
+    status = ds.ds_get_device_status()
+    if status != ds.DS_OK:
+        raise RuntimeError(f"device status after prefill: {ds.strerror(status)}")
+
     traffic = None
     prof = os.path.join(ROOT, "profiles", "topk_traffic.json")
     try:
@@ -386,6 +426,12 @@ def run_ours(args):
             "decode_us_per_step": round(t_dec * 1e3, 2),
             "decode_roofline_us": round(dec_roof_us, 3),
             "decode_frac_of_roofline": round(dec_roof_us / (t_dec * 1e3), 3),
+            "prefill": {"workload": "4096 x 64 x 128 bf16 queries vs 32768 bf16 keys, causal valid_len, k=2048",
+                        "ms_per_call": round(pre_ms, 4), "scorer_ms_per_call": round(pre_score_ms, 4),
+                        "useful_tflop": round(pre_flops / 1e12, 4),
+                        "scorer_tflops": round(pre_flops / (pre_score_ms * 1e-3) / 1e12, 1),
+                        "scorer_frac_of_bf16_peak": round(pre_flops / (pre_score_ms * 1e-3) / 1e12 / tflops_sus, 3),
+                        "bf16_peak_tflops": tflops_sus, "peak_kind": "sustained"},
             "roofline": {"bound": "hbm", "achieved": round(per_launch_gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
                          "frac": round(per_launch_gbs / hbm_gbs, 4), "traffic": traffic,
                          "kernel": TOPK_KERNEL, "peak_source": peak_src},

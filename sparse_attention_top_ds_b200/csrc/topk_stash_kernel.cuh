@@ -156,21 +156,6 @@ __device__ __forceinline__ uint32_t ts_find_bin(const uint32_t* h, int nb, uint3
   return min(ctrl->bcast[0], (uint32_t)(nb - 1));
 }
 
-// Radix digits of the key, most significant first: 12 / 11 / 9 (float32) or
-// 12 / 4 (bfloat16) bits.
-template <class K>
-struct TsDigits;
-template <>
-struct TsDigits<F32Keys> {
-  static constexpr int kCount = 3;
-  __device__ __forceinline__ static int width(int i) { return i == 0 ? 12 : (i == 1 ? 11 : 9); }
-};
-template <>
-struct TsDigits<BF16Keys> {
-  static constexpr int kCount = 2;
-  __device__ __forceinline__ static int width(int i) { return i == 0 ? 12 : 4; }
-};
-
 // Where an exact selection of the kth largest (key, then lower position)
 // cuts: an element is taken when the top bits of its key (key >> kshift)
 // exceed kprefix, or equal it and its position is <= pcut.
@@ -189,38 +174,29 @@ __device__ __forceinline__ bool ts_taken(const TsCut& c, uint32_t key, uint32_t 
 
 // Exact radix select of the kth largest (key, lower position) among the
 // elements that visit(f) hands to f(key, position) (at least kth of them,
-// kth >= 1; positions below 2^24 and distinct).  Radix passes on the key;
-// only if ties at the kth key remain, two 12-bit passes on the complemented
-// positions of the tied elements.  Every thread of the block calls it.
-// When first_ready is set, hist already holds the histogram of the first
-// digit (the top 12 key bits) of those elements.  With start_pass = 1 every
-// visited element has first digit prefix0 and inbin0 elements are visited.
+// kth >= 1; positions below 2^24 and distinct).  Every visited key has top
+// bits ts_top(key, shift0) == prefix0 (shift0 = K::kBits: nothing known), so
+// the passes take 12-bit key digits from bit shift0 down; only if ties at the
+// kth key remain, two 12-bit passes on the complemented positions of the tied
+// elements.  Every thread of the block calls it.
 template <class K, int NT, class Visit>
 __device__ __forceinline__ TsCut ts_select(Visit&& visit, int kth, uint32_t* hist, TsCtrl* ctrl,
-                                           bool first_ready = false, int start_pass = 0, uint32_t prefix0 = 0u,
-                                           uint32_t inbin0 = 0u) {
-  uint32_t prefix = 0;
-  int shift = K::kBits;
+                                           uint32_t prefix0 = 0u, int shift0 = K::kBits) {
+  uint32_t prefix = prefix0;
+  int shift = shift0;
   int krem = kth;
-  if (start_pass == 1) {
-    prefix = prefix0;
-    shift = K::kBits - TsDigits<K>::width(0);
-    if (inbin0 == (uint32_t)kth) return TsCut{prefix, shift, 0xFFFFFFFFu};
-  }
-  for (int pass = start_pass; pass < TsDigits<K>::kCount; ++pass) {
-    const int wd = TsDigits<K>::width(pass);
+  while (shift > 0) {
+    const int wd = shift < 12 ? shift : 12;
     const int sh = shift - wd;
     const uint32_t mask = (1u << wd) - 1u;
-    if (pass > 0 || !first_ready) {
-      for (int i = threadIdx.x; i <= (int)mask; i += NT) hist[i] = 0u;
-      __syncthreads();
-      const uint32_t pf = prefix;
-      const int sf = shift;
-      visit([&](uint32_t key, uint32_t) {
-        if (ts_top(key, sf) == pf) atomicAdd(hist + ((key >> sh) & mask), 1u);
-      });
-      __syncthreads();
-    }
+    for (int i = threadIdx.x; i <= (int)mask; i += NT) hist[i] = 0u;
+    __syncthreads();
+    const uint32_t pf = prefix;
+    const int sf = shift;
+    visit([&](uint32_t key, uint32_t) {
+      if (ts_top(key, sf) == pf) atomicAdd(hist + ((key >> sh) & mask), 1u);
+    });
+    __syncthreads();
     uint32_t above, inbin;
     const uint32_t b = ts_find_bin<NT>(hist, (int)mask + 1, (uint32_t)krem, ctrl, above, inbin);
     krem -= (int)above;
@@ -252,6 +228,40 @@ __device__ __forceinline__ TsCut ts_select(Visit&& visit, int kth, uint32_t* his
   }
   // taken ties: complemented position >= pp << ps
   return TsCut{tkey, 0, ((1u << kTsPosBits) - 1u) - (pp << ps)};
+}
+
+// Block-wide minimum and maximum of one value per thread (every thread calls
+// it and gets both).
+template <int NT>
+__device__ __forceinline__ void ts_block_minmax(uint32_t lo, uint32_t hi, TsCtrl* ctrl, uint32_t& gmin,
+                                                uint32_t& gmax) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+  }
+  if (lane == 0) {
+    ctrl->wtot[warp] = lo;
+    ctrl->wex[warp] = hi;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t a = lane < NT / 32 ? ctrl->wtot[lane] : 0xFFFFFFFFu;
+    uint32_t b = lane < NT / 32 ? ctrl->wex[lane] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      a = min(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+      b = max(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
+    }
+    if (lane == 0) {
+      ctrl->bcast[0] = a;
+      ctrl->bcast[1] = b;
+    }
+  }
+  __syncthreads();
+  gmin = ctrl->bcast[0];
+  gmax = ctrl->bcast[1];
 }
 
 // Hands out n consecutive slots of *counter to each lane of a warp (all 32
@@ -589,7 +599,19 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
       if (i < nc) f(K::key(rr[i]), rp[i]);
     }
   };
-  const TsCut cut = ts_select<K, NT>(visit_stash, kk, hist, ctrl);
+  // the stash's keys share their top bits between its smallest and largest
+  // key: the radix digits start below that common prefix, so the first pass
+  // spreads the stash over many bins
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  visit_stash([&](uint32_t key, uint32_t) {
+    lo = min(lo, key);
+    hi = max(hi, key);
+  });
+  uint32_t gmin, gmax;
+  ts_block_minmax<NT>(lo, hi, ctrl, gmin, gmax);
+  const int common = gmin == gmax ? K::kBits : __clz(gmin ^ gmax) - (32 - K::kBits);
+  const int shift0 = K::kBits - common;
+  const TsCut cut = ts_select<K, NT>(visit_stash, kk, hist, ctrl, ts_top(gmax, shift0), shift0);
   // every selected entry (exactly kk): one warp-level slot allocation per
   // visit; with sorted_index gathered in shared memory first
   uint32_t* sel_pos = hist;
