@@ -46,12 +46,8 @@ struct ScoreCfg {
   static constexpr int kN = NT * HP;                 // accumulator columns per tile
   static constexpr int kNmma = kN < 256 ? kN : 256;  // N of one MMA instruction
   static constexpr int kNumMma = kN / kNmma;
-  static constexpr int kNbuf = kN <= 256 ? 2 : 1;    // TMEM accumulator buffers (per tile)
-  // kN == 512 (8 rows x 64 heads): the accumulator is split into two halves of
-  // 256 columns with their own barriers, so the epilogue of one half overlaps
-  // the MMAs of the other; otherwise whole tiles alternate between 2 buffers.
-  static constexpr bool kSplit = (kN == 512);
-  static constexpr int kEpiPerSlot = kSplit ? 4 : 8;  // epilogue warps releasing one accumulator slot
+  static constexpr int kNbuf = 2;                    // TMEM accumulators: whole tiles alternate between them
+  static constexpr int kEpiPerSlot = 8;              // epilogue warps releasing one accumulator
   static constexpr int kCols = kN * kNbuf;
   static constexpr int kTmemCols = kCols <= 32 ? 32 : (kCols <= 64 ? 64 : (kCols <= 128 ? 128 : (kCols <= 256 ? 256 : 512)));
   static constexpr int kQHalf = kN * 128;            // bytes: kN rows x 64 channels x 2 B
@@ -73,7 +69,7 @@ struct ScoreCfg {
   static constexpr int kNumBars = 5 + 2 * STAGES;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffTmemSlot + 16 + 1024;  // + alignment slack
-  static_assert(kN % 16 == 0 && kN <= 512 && kN % kNmma == 0, "bad tile");
+  static_assert(kN % 16 == 0 && kN <= 256 && kN % kNmma == 0, "bad tile");
   static_assert(HP % 16 == 0 && HP <= 64, "bad head padding");
 };
 
@@ -170,35 +166,25 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
         const int s = i % STAGES, r = i / STAGES;
         if (!mbar_wait_bounded(BAR(C::kBarKFull + s), r & 1, p.status)) break;
         const uint32_t a_base = sbase + C::kOffK + s * C::kStage;
-        // one accumulator slot per MMA group: the two halves (split mode) or
-        // the whole tile in buffer i % 2
-        constexpr int kGroups = C::kSplit ? 2 : 1;
-        constexpr int kMmaPerGroup = C::kNumMma / kGroups;
+        // the whole tile in accumulator buffer i % 2
+        const int slot = i % C::kNbuf;
+        const int use = i / C::kNbuf;
+        if (!mbar_wait_bounded(BAR(C::kBarAEmpty + slot), (use & 1) ^ 1, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_base = tmem_base + (uint32_t)(slot * C::kN);
 #pragma unroll
-        for (int g = 0; g < kGroups; ++g) {
-          const int slot = C::kSplit ? g : (i % C::kNbuf);
-          const int use = C::kSplit ? i : (i / C::kNbuf);
-          if (!mbar_wait_bounded(BAR(C::kBarAEmpty + slot), (use & 1) ^ 1, p.status)) {
-            ok = false;
-            break;
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (uint32_t)(kk & 3) * 32u;  // 16 channels = 32 bytes inside the swizzled row
+          const uint64_t adesc = sw128_kmajor_desc(a_base + (uint32_t)(kk >> 2) * C::kKHalf + koff);
+#pragma unroll
+          for (int j = 0; j < C::kNumMma; ++j) {
+            const uint32_t b_addr = sbase + C::kOffQ + (uint32_t)(kk >> 2) * C::kQHalf +
+                                    (uint32_t)(j * C::kNmma) * 128u + koff;
+            mma_bf16_ss(d_base + (uint32_t)(j * C::kNmma), adesc, sw128_kmajor_desc(b_addr), idesc,
+                        kk > 0 ? 1u : 0u);
           }
-          tc_fence_after();
-          const uint32_t d_base = tmem_base + (uint32_t)((C::kSplit ? 0 : slot) * C::kN);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t koff = (uint32_t)(kk & 3) * 32u;  // 16 channels = 32 bytes inside the swizzled row
-            const uint64_t adesc = sw128_kmajor_desc(a_base + (uint32_t)(kk >> 2) * C::kKHalf + koff);
-#pragma unroll
-            for (int jj = 0; jj < kMmaPerGroup; ++jj) {
-              const int j = g * kMmaPerGroup + jj;
-              const uint32_t b_addr = sbase + C::kOffQ + (uint32_t)(kk >> 2) * C::kQHalf +
-                                      (uint32_t)(j * C::kNmma) * 128u + koff;
-              mma_bf16_ss(d_base + (uint32_t)(j * C::kNmma), adesc, sw128_kmajor_desc(b_addr), idesc,
-                          kk > 0 ? 1u : 0u);
-            }
-          }
-          mma_commit(BAR(C::kBarAFull + slot));
         }
+        mma_commit(BAR(C::kBarAFull + slot));
         mma_commit(BAR(C::kBarKEmpty + s));
       }
     }
@@ -223,9 +209,9 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
       vl[j] = v;
     }
     for (int i = 0; i < nact; ++i) {
-      const int b = C::kSplit ? 0 : (i % C::kNbuf);   // TMEM buffer of this tile
-      const int slot = C::kSplit ? hf : b;             // accumulator slot this warp waits on
-      const int u = C::kSplit ? i : (i / C::kNbuf);
+      const int b = i % C::kNbuf;  // TMEM buffer of this tile
+      const int slot = b;
+      const int u = i / C::kNbuf;
       if (!mbar_wait_bounded(BAR(C::kBarAFull + slot), u & 1, p.status)) break;  // status records the timeout
       tc_fence_after();
       const int s = (tile_lo + i) * 128 + row;

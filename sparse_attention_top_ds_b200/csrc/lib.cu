@@ -315,7 +315,6 @@ static cudaError_t indexer_setup() {
   cudaError_t e = set_score_smem<1, 64, 4>();
   if (e == cudaSuccess) e = set_score_smem<2, 64, 4>();
   if (e == cudaSuccess) e = set_score_smem<4, 64, 4>();
-  if (e == cudaSuccess) e = set_score_smem<8, 64, 2>();
   if (e == cudaSuccess) e = set_score_smem<8, 32, 4>();
   if (e == cudaSuccess) e = set_score_smem<8, 16, 4>();
   if (e == cudaSuccess)
@@ -420,8 +419,10 @@ static int score_enqueue(const void* q, const void* kc, const float* w, int B, i
   if (H > 32) {
     if (B == 1) return launch_score<1, 64, 4>(q, kc, w, B, H, S, vl, out, st, s);
     if (B == 2) return launch_score<2, 64, 4>(q, kc, w, B, H, S, vl, out, st, s);
+    // 5..8 rows: two rows per CTA (measured faster than eight per CTA, whose
+    // 128 KiB query tile every CTA must load)
     if (B <= 4 || B > 8) return launch_score<4, 64, 4>(q, kc, w, B, H, S, vl, out, st, s);
-    return launch_score<8, 64, 2>(q, kc, w, B, H, S, vl, out, st, s);
+    return launch_score<2, 64, 4>(q, kc, w, B, H, S, vl, out, st, s);
   }
   if (H > 16) return launch_score<8, 32, 4>(q, kc, w, B, H, S, vl, out, st, s);
   return launch_score<8, 16, 4>(q, kc, w, B, H, S, vl, out, st, s);
