@@ -41,7 +41,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 1024 * 1024
 
 SAMPLING = dict(batch=64, n=129280, ks=(1024, 64))
-# ds_topk runs the one-pass stash kernel for >= 32 rows (the cluster kernel below)
+# ds_topk runs the one-pass stash kernel for >= 64 rows (the cluster kernel below)
 TOPK_KERNEL = "topk_stash_kernel<F32Keys, 1024>"
 DECODE = dict(batch=8, heads=64, d=128, S=32768, k=1024)
 PREFILL = dict(k=2048)

@@ -140,8 +140,10 @@ static bool choose_topk_shape(int batch, int n, int num_sms, TopkShape* out) {
   slice = (slice + 7) / 8 * 8;
   out->cluster = C;
   out->slice = slice;
+  // 512 threads measured faster for up to 16 rows, 256 for more
+  out->threads = batch <= 16 ? 512 : 256;
   const char* nt = getenv("DS_TOPK_THREADS");      // tuning sweeps only
-  out->threads = (nt && atoi(nt) == 256) ? 256 : 512;  // 512 measured faster on every few-row shape
+  if (nt && (atoi(nt) == 256 || atoi(nt) == 512)) out->threads = atoi(nt);
   return true;
 }
 
@@ -254,15 +256,15 @@ static int topk_stash_enqueue(const void* scores, int batch, int n, int k, int d
   return e == cudaSuccess ? DS_OK : DS_ERR_CUDA;
 }
 
-// Two kernels: with many rows (>= 32) the one-pass stash kernel, whose rows
-// fill the SMs with one or two CTAs each; with few rows the cluster kernel
+// Two kernels: with many rows (>= 64) the one-pass stash kernel, whose rows
+// fill the SMs with one or two CTAs each; with fewer rows the cluster kernel
 // (topk_kernel.cuh), which spreads a row over up to 16 CTAs and has the
-// shorter fixed chain of steps.  DS_TOPK_KERNEL=stash / cluster picks one
-// regardless (tests and comparisons).
+// shorter fixed chain of steps (both measured on each side of the boundary).
+// DS_TOPK_KERNEL=stash / cluster picks one regardless (tests and comparisons).
 static int topk_enqueue(const void* scores, int batch, int n, int k, int dtype, const int32_t* valid_len,
                         int32_t* out_idx, void* out_val, int return_value, int sorted_index, cudaStream_t st,
                         DeviceState* s) {
-  bool stash = batch >= 32;
+  bool stash = batch >= 64;
   const char* pick = getenv("DS_TOPK_KERNEL");
   if (pick && strcmp(pick, "stash") == 0) stash = true;
   if (pick && strcmp(pick, "cluster") == 0) stash = false;
