@@ -91,9 +91,7 @@ static int device_state(DeviceState** out) {
         e = cudaFuncSetAttribute(topk_cluster_kernel<BF16Keys, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(topk_cluster_kernel<BF16Keys, 512>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
-      if (e == cudaSuccess) e = set_stash_smem<256>(smem_max);
-      if (e == cudaSuccess) e = set_stash_smem<512>(smem_max);
-      if (e == cudaSuccess) e = set_stash_smem<1024>(smem_max);
+      if (e == cudaSuccess) e = set_stash_smem<kTsThreads>(smem_max);
       if (e == cudaSuccess) e = indexer_setup();
       if (e != cudaSuccess) return DS_ERR_CUDA;
       g_max_cluster = topk_cluster16_ok() ? 16 : 8;
@@ -239,20 +237,8 @@ static int topk_stash_enqueue(const void* scores, int batch, int n, int k, int d
   set_pdl(attr[1]);
   cfg.attrs = attr;
   cfg.numAttrs = pdl_on() ? 2 : 1;
-  int nt = kTsThreads;
-  const char* fnt = getenv("DS_TOPK_NT");  // tuning sweeps only
-  if (fnt && (atoi(fnt) == 256 || atoi(fnt) == 512 || atoi(fnt) == 1024)) nt = atoi(fnt);
-  cfg.blockDim = dim3((unsigned)nt, 1, 1);
-  cudaError_t e;
-  if (nt == 256)
-    e = dtype == DS_F32 ? cudaLaunchKernelEx(&cfg, topk_stash_kernel<F32Keys, 256>, p)
-                        : cudaLaunchKernelEx(&cfg, topk_stash_kernel<BF16Keys, 256>, p);
-  else if (nt == 1024)
-    e = dtype == DS_F32 ? cudaLaunchKernelEx(&cfg, topk_stash_kernel<F32Keys, 1024>, p)
-                        : cudaLaunchKernelEx(&cfg, topk_stash_kernel<BF16Keys, 1024>, p);
-  else
-    e = dtype == DS_F32 ? cudaLaunchKernelEx(&cfg, topk_stash_kernel<F32Keys, 512>, p)
-                        : cudaLaunchKernelEx(&cfg, topk_stash_kernel<BF16Keys, 512>, p);
+  const cudaError_t e = dtype == DS_F32 ? cudaLaunchKernelEx(&cfg, topk_stash_kernel<F32Keys, kTsThreads>, p)
+                                        : cudaLaunchKernelEx(&cfg, topk_stash_kernel<BF16Keys, kTsThreads>, p);
   return e == cudaSuccess ? DS_OK : DS_ERR_CUDA;
 }
 
