@@ -203,3 +203,21 @@ def test_argument_errors(cuda_device):
     too_long = torch.zeros((1, (1 << 24) + 8), dtype=torch.float32, device="cuda")
     with pytest.raises(ds.DsError):
         ds.ds_topk(too_long, 10)
+
+
+def test_scores_produced_by_the_previous_kernel(cuda_device):
+    # ds_topk may start while the previous kernel on the stream finishes
+    # (programmatic dependent launch); it must still read that kernel's
+    # finished output: here the scores come from a PyTorch kernel launched
+    # right before, and each call's selection is checked against the oracle
+    g = torch.Generator(device="cuda").manual_seed(11)
+    idx_out = torch.empty((64, 256), dtype=torch.int32, device="cuda")
+    for it in range(4):
+        base = torch.randn((64, 40000), device="cuda", generator=g)
+        scores = base * 3.0 + float(it)          # the producing kernel
+        idx, val = ds.ds_topk(scores, 256, out_idx=idx_out)
+        torch.cuda.synchronize()
+        assert ds.ds_get_device_status() == ds.DS_OK
+        raw = scores.cpu().numpy()
+        ref_idx, _ = oracle.topk_rows(raw, "f32", 256)
+        assert_topk_exact(idx.cpu().numpy(), bits_of(val), raw.view(np.uint32), ref_idx, 256, False)
