@@ -9,6 +9,9 @@ seeded input:
     and indices, unsorted;
   * the decode indexer + top-k (8 query rows x 64 heads x 128 bf16 against one
     bf16 key cache of 32768 positions, valid_len ~ U{4096..32768}, k = 1024).
+Reported beside it: the prefill indexer + top-k, and the sparse attention that
+consumes the selection (8 tokens x 128 heads x 512 over k = 1024 selected rows
+plus a window of 128, L2 flushed before each call).
 The headline value is the top-k effective HBM bandwidth (algorithmic bytes /
 device time, GB/s); the decode indexer + top-k time is reported in
 microseconds per decode step beside it.  Inputs rotate through enough copies
@@ -45,6 +48,8 @@ SAMPLING = dict(batch=64, n=129280, ks=(1024, 64))
 TOPK_KERNEL = "topk_stash_kernel<F32Keys, 1024>"
 DECODE = dict(batch=8, heads=64, d=128, S=32768, k=1024)
 PREFILL = dict(k=2048)
+ATTENTION = dict(batch=8, heads=128, d=512, T=32768, k=1024, W=128)
+ATTN_CALLS = 40
 
 
 def load_peaks():
@@ -69,6 +74,19 @@ def decode_bytes_flops(vl, heads, d, k):
     B = len(vl)
     bytes_ = maxvl * d * 2 + B * heads * d * 2 + B * heads * 4 + B * 4 + B * k * 4
     flops = 2 * heads * d * int(np.sum(vl))
+    return bytes_, flops
+
+
+def attention_bytes_flops(idx, T, win_len, heads, d, k):
+    """Algorithmic bytes and FLOPs of one sparse-attention call: every attended
+    row read once (it is both key and value), queries read and outputs (bf16
+    out, float32 lse) written once, the slots and the sink read once; two
+    products of 2 * heads * d FLOPs per attended row."""
+    idx = np.asarray(idx)
+    rows = int(((idx >= 0) & (idx < T)).sum()) + int(np.sum(win_len))
+    B = idx.shape[0]
+    bytes_ = rows * d * 2 + 2 * B * heads * d * 2 + B * heads * 4 + B * k * 4 + heads * 4 + B * 4
+    flops = 4.0 * heads * d * rows
     return bytes_, flops
 
 
@@ -390,6 +408,60 @@ def run_ours(args):
     if status != ds.DS_OK:
         raise RuntimeError(f"device status after prefill: {ds.strerror(status)}")
 
+    # ---- sparse attention over the selected rows (the step that consumes the
+    # selection), beside the headline: 8 tokens x 128 heads x d = 512 against
+    # a 32768-row cache per batch row, k = 1024 slots plus a window of 128.
+    # L2 is flushed (a 256 MiB write) before every timed call, so the gathered
+    # rows come from HBM as they do after the selection step.
+    A = ATTENTION
+    aa = inputs.attention(seed=inputs.SEED_ATTENTION + rank, batch=A["batch"], heads=A["heads"], d=A["d"],
+                          T=A["T"], k=A["k"], W=A["W"])
+    a_q = torch.from_numpy(aa["q"].view(np.int16)).view(torch.bfloat16).to(dev)
+    a_kv = torch.from_numpy(aa["kv"].view(np.int16)).view(torch.bfloat16).to(dev)
+    a_win = torch.from_numpy(aa["win"].view(np.int16)).view(torch.bfloat16).to(dev)
+    a_idx = torch.from_numpy(aa["idx"]).to(dev)
+    a_wl = torch.from_numpy(aa["win_len"]).to(dev)
+    a_sink = torch.from_numpy(aa["sink"]).to(dev)
+    a_out = torch.empty((A["batch"], A["heads"], A["d"]), dtype=torch.bfloat16, device=dev)
+    a_lse = torch.empty((A["batch"], A["heads"]), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def attn_call():
+        ds.ds_sparse_attention(a_q, a_kv, a_idx, win=a_win, win_len=a_wl, sink=a_sink, out=a_out, lse=a_lse)
+
+    for _ in range(3):
+        attn_call()
+    torch.cuda.synchronize()
+    barrier()
+    a_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(ATTN_CALLS)]
+    for i in range(ATTN_CALLS):
+        flush.fill_(float(i))
+        a_ev[i][0].record(stream)
+        attn_call()
+        a_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    attn_us = sum(e0.elapsed_time(e1) for e0, e1 in a_ev) / ATTN_CALLS * 1e3
+    (attn_us,) = max_over_ranks([attn_us], dev)
+    del flush
+    status = ds.ds_get_device_status()
+    if status != ds.DS_OK:
+        raise RuntimeError(f"device status after attention: {ds.strerror(status)}")
+    abytes, aflops = attention_bytes_flops(aa["idx"], A["T"], aa["win_len"], A["heads"], A["d"], A["k"])
+    a_t_hbm = abytes / (hbm_gbs * 1e9) * 1e6
+    a_t_tc = aflops / (tflops * 1e12) * 1e6
+    attention = {
+        "workload": "8 tokens x 128 heads x d=512 bf16 queries; per-row bf16 cache of 32768 x 512; k=1024 "
+                    "selected rows + window of 128 + per-head sink; out bf16 + lse f32; L2 flushed per call",
+        "us_per_call": round(attn_us, 2),
+        "roofline_us": round(max(a_t_hbm, a_t_tc), 3),
+        "bound": "hbm" if a_t_hbm >= a_t_tc else "tensor",
+        "frac_of_roofline": round(max(a_t_hbm, a_t_tc) / attn_us, 3),
+        "achieved_gbs": round(abytes / (attn_us * 1e-6) / 1e9, 1),
+        "achieved_tflops": round(aflops / (attn_us * 1e-6) / 1e12, 1),
+        "algorithmic_bytes": int(abytes), "flops": int(aflops),
+        "peaks": {"hbm_gbs": hbm_gbs, "bf16_tflops": tflops, "kind": "burst"},
+    }
+
     traffic = None
     prof = os.path.join(ROOT, "profiles", "topk_traffic.json")
     try:
@@ -432,6 +504,7 @@ def run_ours(args):
                         "scorer_tflops": round(pre_flops / (pre_score_ms * 1e-3) / 1e12, 1),
                         "scorer_frac_of_bf16_peak": round(pre_flops / (pre_score_ms * 1e-3) / 1e12 / tflops_sus, 3),
                         "bf16_peak_tflops": tflops_sus, "peak_kind": "sustained"},
+            "sparse_attention": attention,
             "roofline": {"bound": "hbm", "achieved": round(per_launch_gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
                          "frac": round(per_launch_gbs / hbm_gbs, 4), "traffic": traffic,
                          "kernel": TOPK_KERNEL, "peak_source": peak_src},

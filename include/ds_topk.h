@@ -2,7 +2,7 @@
  * ds_topk.h -- C ABI of libdstopk.so, the selection step of DeepSeek-style
  * sparse attention on B200 (sm_100a).
  *
- * Two operations, as described on the pages this library follows:
+ * Three operations, as described on the pages this library follows:
  *
  *  - Row-wise top-k of given scores (DeepSelect hub page, use-case paragraphs:
  *    pick the top-k positions of every score row; bfloat16 rows for the
@@ -15,6 +15,10 @@
  *        score[t,s] = sum_h w[t,h] * max(0, q[t,h,:] . k[s,:])
  *    over a 128-channel bfloat16 key cache shared by all rows, then the k
  *    highest-scoring positions of each row.
+ *
+ *  - The attention that consumes the selection (the same pull request, steps
+ *    table row 4): multi-query softmax attention of every query head over
+ *    the selected compressed KV rows plus a sliding window of recent rows.
  *
  * Conventions shared by every entry point
  *  - All tensor arguments are DEVICE pointers to caller-owned memory, row-major
@@ -31,9 +35,10 @@
  *    equal.  Positions s >= valid_len[row] are never selected.  When a row
  *    has fewer than k eligible positions, the missing slots hold index -1 and
  *    value / score -inf.
- *  - The library owns only scratch memory: ds_indexer_topk allocates a
- *    per-device, grow-only buffer with cudaMalloc on first use (so make the
- *    first call outside CUDA-graph capture); ds_release frees it.
+ *  - The library owns only scratch memory: ds_indexer_topk and
+ *    ds_sparse_attention each allocate a per-device, grow-only buffer with
+ *    cudaMalloc on first use (so make the first call outside CUDA-graph
+ *    capture); ds_release frees them.
  *  - Calls on different streams may run concurrently, except that calls of
  *    ds_indexer_topk on one device share the scratch buffer and must be
  *    ordered on one stream.
@@ -62,6 +67,9 @@ typedef enum { DS_F32 = 0, DS_BF16 = 1 } ds_dtype;
 #define DS_MAX_K 2048            /* largest k of either operation */
 #define DS_INDEXER_DIM 128       /* indexer channels d (fixed) */
 #define DS_INDEXER_MAX_HEADS 64  /* largest number of indexer heads */
+#define DS_ATTN_MAX_DIM 512      /* largest head_dim of ds_sparse_attention */
+#define DS_ATTN_MAX_WINDOW 4096  /* largest sliding window of ds_sparse_attention */
+#define DS_ATTN_MAX_HEADS 4096   /* largest number of query heads of ds_sparse_attention */
 
 /*
  * ds_topk -- top-k of every row of a [batch, n] score matrix.
@@ -161,6 +169,64 @@ int ds_indexer_topk_noalloc(const void* q, const void* kcache, const float* w,
                             int batch, int heads, int d, int S,
                             const int32_t* valid_len, int k,
                             int32_t* out_idx, float* out_score, void* stream);
+
+/*
+ * ds_sparse_attention -- multi-query decode attention over the selected
+ * compressed rows plus a sliding window.
+ *   (NKI pull request "Add DeepSeek-V4 CSA attention kernels", "How the
+ *    algorithm works": the attention reads only the selected compressed
+ *    positions plus a local window, and steps table row 4 "Concatenate and
+ *    attend"; "The top-k on the GPSIMD engine", last paragraph: K and V are
+ *    the same embedding; "Launching a full block": the window cache
+ *    [B, W, head_dim] and the compressed cache [B, T_c, head_dim].)
+ *
+ * For batch row b and head h, with r over the attended rows -- the cache rows
+ * kv_b[idx[b, j]] of every slot j with 0 <= idx[b, j] < T, then the window
+ * rows win[b, i] for i < win_len[b] -- each row serving as key and value:
+ *     z[r]        = scale * (q[b, h, :] . row_r)
+ *     out[b, h, :] = sum_r e^z[r] row_r / (sum_r e^z[r] + e^sink[h])
+ *     lse[b, h]    = log(sum_r e^z[r] + e^sink[h])
+ * The sink terms are absent when sink is NULL.  With nothing attended and no
+ * sink, out is 0 and lse is -inf.
+ *
+ * q            device bfloat16 [batch, heads, d]; 16-byte aligned.
+ * kv           device bfloat16: batch row b's compressed cache is the T rows of
+ *              d elements that start kv_batch_stride * b rows after kv;
+ *              16-byte aligned.
+ * kv_batch_stride  rows from one batch row's cache to the next, >= 0: 0 for one
+ *              cache shared by every batch row, T for a [batch, T, d] array.
+ * T            rows of each cache, >= 1.
+ * idx          device int32 [batch, k]: the selected rows (for instance the
+ *              output of ds_indexer_topk).  Slots outside [0, T), such as the
+ *              -1 padding of the top-k, are skipped; every other slot is
+ *              attended, so a repeated index counts once per slot.
+ * k            slots per batch row, 0 <= k <= DS_MAX_K; idx may be NULL if k = 0.
+ * win          device bfloat16 [batch, W, d] or NULL (then W must be 0);
+ *              16-byte aligned.
+ * W            window rows per batch row, 0 <= W <= DS_ATTN_MAX_WINDOW.
+ * win_len      device int32 [batch] or NULL (= W): window rows
+ *              0 .. min(max(win_len[b], 0), W) - 1 are attended.
+ * sink         device float32 [heads] or NULL: one logit per head.
+ * batch        1 .. 65535;  heads 1 .. DS_ATTN_MAX_HEADS;
+ * d            a multiple of 64, 64 <= d <= DS_ATTN_MAX_DIM.
+ * scale        finite score factor (1/sqrt(d) for the usual attention).
+ * out          device bfloat16 [batch, heads, d]; 16-byte aligned.
+ * lse          device float32 [batch, heads] or NULL (natural logarithm).
+ * Inputs are expected to be finite.  The products q . row are bf16 x bf16
+ * accumulated in float32 on the tensor cores; the softmax is float32 with its
+ * weights rounded to bfloat16 for the weighted sum (also a tensor-core
+ * product), and the normaliser sums those rounded weights; out is rounded to
+ * the nearest bfloat16.
+ * Uses a scratch buffer of its own (per device, grow-only, allocated with
+ * cudaMalloc on first use and by calls larger than any before, so make such
+ * calls outside CUDA-graph capture; freed by ds_release): calls of
+ * ds_sparse_attention on one device must be ordered on one stream.
+ * Returns DS_OK, DS_ERR_ARG, DS_ERR_UNSUPPORTED, DS_ERR_NOMEM or DS_ERR_CUDA.
+ */
+int ds_sparse_attention(const void* q, const void* kv, int64_t kv_batch_stride, int T,
+                        const int32_t* idx, int k, const void* win, int W, const int32_t* win_len,
+                        const float* sink, int batch, int heads, int d, float scale,
+                        void* out, float* lse, void* stream);
 
 /*
  * ds_get_device_status -- synchronise `stream`, then return and clear the

@@ -14,6 +14,10 @@ selection step computes, in float64:
                     use-case paragraphs: lightning indexer at topk=512 in
                     bfloat16, sampling over a ~128K vocabulary in float32, and
                     the ``sorted_index`` / ``return_value`` options).
+* ``attention``  -- multi-query softmax attention over the selected compressed
+                    rows plus a sliding window (NKI pull request, steps table
+                    row 4 "Concatenate and attend"), with an optional per-head
+                    attention sink.
 * ``indexer``    -- the lightning-indexer score
                     ``score[t,s] = sum_h w[t,h] * max(0, q[t,h,:] . k[s,:])``
                     (NKI pull request "Add DeepSeek-V4 CSA attention kernels",
@@ -28,8 +32,9 @@ and invariants; no function here is "parity unpinned".
 from .encoding import decode_bf16, decode_f32, NEG_INF_BF16, NEG_INF_F32
 from .topk import topk_rows, topk_row
 from .indexer import indexer_scores, indexer_topk
+from .attention import sparse_attention
 
 __all__ = [
     "decode_bf16", "decode_f32", "NEG_INF_BF16", "NEG_INF_F32",
-    "topk_rows", "topk_row", "indexer_scores", "indexer_topk",
+    "topk_rows", "topk_row", "indexer_scores", "indexer_topk", "sparse_attention",
 ]

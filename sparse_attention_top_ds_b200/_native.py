@@ -24,6 +24,9 @@ DS_ERR_NOMEM = -5
 DS_MAX_K = 2048
 DS_INDEXER_DIM = 128
 DS_INDEXER_MAX_HEADS = 64
+DS_ATTN_MAX_DIM = 512
+DS_ATTN_MAX_WINDOW = 4096
+DS_ATTN_MAX_HEADS = 4096
 
 _lib = None
 
@@ -57,6 +60,9 @@ def load():
     lib.ds_indexer_topk.restype = i32
     lib.ds_indexer_topk_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32p, i32, vp, vp, vp]
     lib.ds_indexer_topk_noalloc.restype = i32
+    lib.ds_sparse_attention.argtypes = [vp, vp, ctypes.c_int64, i32, i32p, i32, vp, i32, i32p, vp,
+                                        i32, i32, i32, ctypes.c_float, vp, vp, vp]
+    lib.ds_sparse_attention.restype = i32
     lib.ds_get_device_status.argtypes = [vp]
     lib.ds_get_device_status.restype = i32
     lib.ds_strerror.argtypes = [i32]
@@ -95,6 +101,12 @@ def ds_indexer_topk_noalloc_raw(q, kcache, w, batch, heads, d, S, valid_len, k, 
     """The allocation-free variant (score rows in the library's fixed array)."""
     return load().ds_indexer_topk_noalloc(q, kcache, w, batch, heads, d, S, valid_len, k, out_idx, out_score,
                                           stream)
+
+
+def ds_sparse_attention_raw(q, kv, kv_batch_stride, T, idx, k, win, W, win_len, sink, batch, heads, d, scale,
+                            out, lse, stream):
+    return load().ds_sparse_attention(q, kv, int(kv_batch_stride), T, idx, k, win, W, win_len, sink,
+                                      batch, heads, d, float(scale), out, lse, stream)
 
 
 def ds_get_device_status(stream=None):
@@ -213,3 +225,65 @@ def ds_indexer_topk(q, kcache, w, k, valid_len=None, return_score=False,
                                  _ptr(out_score) if return_score else None, _stream_ptr(stream))
     _check(rc, "ds_indexer_topk")
     return out_idx, (out_score if return_score else None)
+
+
+def ds_sparse_attention(q, kv, idx, scale=None, win=None, win_len=None, sink=None, return_lse=False,
+                        out=None, lse=None, stream=None):
+    """Multi-query attention of every query head over the selected cache rows
+    plus a sliding window.
+
+    q    bf16 [batch, heads, d];  kv  bf16 [T, d] (one cache for every batch
+    row) or [batch, T, d];  idx  int32 [batch, k] or None (window only);
+    win  bf16 [batch, W, d] or None;  win_len  int32 [batch] or None (= W);
+    sink float32 [heads] or None;  scale  default 1/sqrt(d).
+    Returns out bf16 [batch, heads, d], or (out, lse float32 [batch, heads]).
+    """
+    import math
+    import torch
+    _require(q, torch.bfloat16, "q")
+    dev = q.device
+    _require(kv, torch.bfloat16, "kv", dev)
+    if q.dim() != 3:
+        raise ValueError("q must be [batch, heads, d]")
+    batch, heads, d = q.shape
+    if kv.dim() == 2:
+        T, stride = kv.shape[0], 0
+    elif kv.dim() == 3 and kv.shape[0] == batch:
+        T, stride = kv.shape[1], kv.shape[1]
+    else:
+        raise ValueError("kv must be [T, d] or [batch, T, d]")
+    if kv.shape[-1] != d:
+        raise ValueError("kv and q differ in d")
+    k = 0
+    if idx is not None:
+        _require(idx, torch.int32, "idx", dev)
+        if idx.dim() != 2 or idx.shape[0] != batch:
+            raise ValueError("idx must be [batch, k]")
+        k = idx.shape[1]
+    W = 0
+    if win is not None:
+        _require(win, torch.bfloat16, "win", dev)
+        if win.dim() != 3 or win.shape[0] != batch or win.shape[2] != d:
+            raise ValueError("win must be [batch, W, d]")
+        W = win.shape[1]
+    if win_len is not None:
+        _require(win_len, torch.int32, "win_len", dev)
+    if sink is not None:
+        _require(sink, torch.float32, "sink", dev)
+        if sink.numel() != heads:
+            raise ValueError("sink must hold one logit per head")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((batch, heads, d), dtype=torch.bfloat16, device=dev)
+    _require(out, torch.bfloat16, "out", dev)
+    if return_lse and lse is None:
+        lse = torch.empty((batch, heads), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _require(lse, torch.float32, "lse", dev)
+    with torch.cuda.device(dev):
+        rc = ds_sparse_attention_raw(_ptr(q), _ptr(kv), stride, T, _ptr(idx), k, _ptr(win), W, _ptr(win_len),
+                                     _ptr(sink), batch, heads, d, scale, _ptr(out), _ptr(lse),
+                                     _stream_ptr(stream))
+    _check(rc, "ds_sparse_attention")
+    return (out, lse) if return_lse else out

@@ -1,6 +1,7 @@
 // lib.cu -- the C ABI of libdstopk.so (declared in include/ds_topk.h):
 // argument checks, launch-shape choice and kernel launches.  One translation
 // unit holds every kernel, so device symbols (the status word) resolve here.
+#include <algorithm>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -17,6 +18,7 @@
 #include "indexer_kernel.cuh"
 #include "decode_kernel.cuh"
 #include "rowcluster_kernel.cuh"
+#include "attention_kernel.cuh"
 
 namespace dstopk {
 
@@ -38,6 +40,8 @@ struct DeviceState {
   int dec_max_blocks = 0;        // co-resident CTAs of the fused decode kernel
   int rc_cluster = 0;            // row-per-cluster indexer + top-k: CTAs per row (0: unavailable)
   int rc_active = 0;             // clusters of that size the device runs at once
+  void* attn_scratch = nullptr;  // sparse attention: per-chunk partial results, grow-only
+  size_t attn_scratch_bytes = 0;
 };
 
 static std::mutex g_mu;
@@ -311,6 +315,9 @@ static cudaError_t indexer_setup() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(indexer_topk_rowcluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              RcSmem::kBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(sparse_attn_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnSmem::bytes(kAttnMaxD));
   return e;
 }
 
@@ -571,6 +578,119 @@ static void* get_scratch(DeviceState* s, size_t bytes) {
   return p;
 }
 
+// ---- sparse attention over the selected rows
+
+// Queries [rows][D] bf16 in boxes of 64 channels x 128 heads, 128-byte swizzle.
+static bool encode_attn_q(const void* q, long long rows, int D, CUtensorMap* tq) {
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t str[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kAttnHeads};
+  cuuint32_t one[2] = {1, 1};
+  const CUresult r = g_encode(tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, str, box, one,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Partial results of one call stay below this; larger batches run in pieces.
+constexpr size_t kAttnScratchCap = size_t(512) << 20;
+
+static void* get_attn_scratch(DeviceState* s, size_t bytes) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (s->attn_scratch_bytes >= bytes) return s->attn_scratch;
+  if (s->attn_scratch) cudaFree(s->attn_scratch);
+  s->attn_scratch = nullptr;
+  s->attn_scratch_bytes = 0;
+  void* p = nullptr;
+  if (cudaMalloc(&p, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  s->attn_scratch = p;
+  s->attn_scratch_bytes = bytes;
+  return p;
+}
+
+static int attention_enqueue(const uint16_t* q, const uint16_t* kv, long long kv_bstride_rows, int T,
+                             const int32_t* idx, int k, const uint16_t* win, int W, const int32_t* win_len,
+                             const float* sink, int B, int H, int D, float scale, uint16_t* out, float* lse,
+                             cudaStream_t st, DeviceState* s) {
+  const int HT = (H + kAttnHeads - 1) / kAttnHeads;
+  const int NS = (k + W + kAttnRows - 1) / kAttnRows;
+  const size_t opart_row = (size_t)HT * NS * (size_t)D * kAttnHeads * sizeof(float);
+  const size_t ml_row = (size_t)HT * NS * kAttnHeads * sizeof(float2);
+  int per = B;
+  if (NS > 0 && (opart_row + ml_row) * (size_t)B > kAttnScratchCap)
+    per = (int)std::max<size_t>(1, kAttnScratchCap / (opart_row + ml_row));
+  float* opart = nullptr;
+  float2* ml = nullptr;
+  if (NS > 0) {
+    uint8_t* base = static_cast<uint8_t*>(get_attn_scratch(s, (opart_row + ml_row) * (size_t)per));
+    if (!base) return DS_ERR_NOMEM;
+    opart = reinterpret_cast<float*>(base);
+    ml = reinterpret_cast<float2*>(base + opart_row * (size_t)per);
+  }
+  const float kLog2e = 1.4426950408889634f;
+  for (int b0 = 0; b0 < B; b0 += per) {
+    const int nb = std::min(per, B - b0);
+    if (NS > 0) {
+      CUtensorMap tq;
+      if (!encode_attn_q(q + (size_t)b0 * H * D, (long long)nb * H, D, &tq)) return DS_ERR_ARG;
+      AttnParams p;
+      p.kv = kv + (size_t)b0 * (size_t)kv_bstride_rows * D;
+      p.kv_bstride = kv_bstride_rows * (long long)D;
+      p.win = win ? win + (size_t)b0 * W * D : nullptr;
+      p.idx = idx ? idx + (size_t)b0 * k : nullptr;
+      p.win_len = win_len ? win_len + b0 : nullptr;
+      p.opart = opart;
+      p.ml = ml;
+      p.status = s->status;
+      p.T = T;
+      p.k = k;
+      p.W = W;
+      p.B = nb;
+      p.H = H;
+      p.D = D;
+      p.HT = HT;
+      p.NS = NS;
+      p.scale_log2 = scale * kLog2e;
+      cudaLaunchConfig_t cfg;
+      memset(&cfg, 0, sizeof(cfg));
+      cfg.gridDim = dim3((unsigned)NS, (unsigned)HT, (unsigned)nb);
+      cfg.blockDim = dim3(kAttnThreads, 1, 1);
+      cfg.dynamicSmemBytes = (size_t)AttnSmem::bytes(D);
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      set_pdl(attr[0]);
+      cfg.attrs = attr;
+      cfg.numAttrs = pdl_on() ? 1 : 0;
+      if (cudaLaunchKernelEx(&cfg, sparse_attn_partial_kernel, tq, p) != cudaSuccess) return DS_ERR_CUDA;
+    }
+    AttnCombineParams c;
+    c.opart = opart;
+    c.ml = ml;
+    c.sink = sink;
+    c.out = out + (size_t)b0 * H * D;
+    c.lse = lse ? lse + (size_t)b0 * H : nullptr;
+    c.B = nb;
+    c.H = H;
+    c.D = D;
+    c.HT = HT;
+    c.NS = NS;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)(D / 64), (unsigned)((H + 31) / 32), (unsigned)nb);
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    set_pdl(attr[0]);
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_on() ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, sparse_attn_combine_kernel, c) != cudaSuccess) return DS_ERR_CUDA;
+  }
+  return DS_OK;
+}
+
 }  // namespace dstopk
 
 using namespace dstopk;
@@ -618,12 +738,15 @@ extern "C" void ds_release(void) {
   int cur = -1;
   if (cudaGetDevice(&cur) != cudaSuccess) cur = -1;
   for (int d = 0; d < kMaxDevices; ++d) {
-    if (g_dev[d].scratch || g_dev[d].dec_ctl || g_dev[d].dec_cand) {
+    if (g_dev[d].scratch || g_dev[d].dec_ctl || g_dev[d].dec_cand || g_dev[d].attn_scratch) {
       if (cudaSetDevice(d) == cudaSuccess) {
         if (g_dev[d].scratch) cudaFree(g_dev[d].scratch);
         if (g_dev[d].dec_ctl) cudaFree(g_dev[d].dec_ctl);
         if (g_dev[d].dec_cand) cudaFree(g_dev[d].dec_cand);
+        if (g_dev[d].attn_scratch) cudaFree(g_dev[d].attn_scratch);
       }
+      g_dev[d].attn_scratch = nullptr;
+      g_dev[d].attn_scratch_bytes = 0;
       g_dev[d].scratch = nullptr;
       g_dev[d].scratch_bytes = 0;
       g_dev[d].dec_ctl = nullptr;
@@ -721,4 +844,25 @@ extern "C" int ds_indexer_topk_noalloc(const void* q, const void* kcache, const 
   rc = score_enqueue(q, kcache, w, batch, heads, S, valid_len, scores, st, s);
   if (rc != DS_OK) return rc;
   return topk_enqueue(scores, batch, S, k, DS_F32, valid_len, out_idx, out_score, out_score != nullptr, 0, st, s);
+}
+
+extern "C" int ds_sparse_attention(const void* q, const void* kv, int64_t kv_batch_stride, int T, const int32_t* idx,
+                                   int k, const void* win, int W, const int32_t* win_len, const float* sink,
+                                   int batch, int heads, int d, float scale, void* out, float* lse, void* stream) {
+  auto misaligned = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; };
+  if (!q || !kv || !out || batch <= 0 || batch > 65535 || heads <= 0 || heads > DS_ATTN_MAX_HEADS) return DS_ERR_ARG;
+  if (d < 64 || d > DS_ATTN_MAX_DIM || d % 64 != 0 || T <= 0 || kv_batch_stride < 0) return DS_ERR_ARG;
+  if (k < 0 || k > DS_MAX_K || (k > 0 && !idx) || W < 0 || W > DS_ATTN_MAX_WINDOW || (W > 0 && !win))
+    return DS_ERR_ARG;
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return DS_ERR_ARG;
+  if (misaligned(q, 16) || misaligned(kv, 16) || misaligned(out, 16) || (win && misaligned(win, 16)) ||
+      (idx && misaligned(idx, 4)) || (win_len && misaligned(win_len, 4)) || (sink && misaligned(sink, 4)) ||
+      (lse && misaligned(lse, 4)))
+    return DS_ERR_ARG;
+  DeviceState* s = nullptr;
+  const int rc = device_state(&s);
+  if (rc != DS_OK) return rc;
+  return attention_enqueue(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(kv), (long long)kv_batch_stride,
+                           T, idx, k, static_cast<const uint16_t*>(win), W, win_len, sink, batch, heads, d, scale,
+                           static_cast<uint16_t*>(out), lse, static_cast<cudaStream_t>(stream), s);
 }

@@ -51,8 +51,24 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
   return d;
 }
 
+// Descriptor of an MN-major operand in the same 128-byte-swizzled layout:
+// 64 consecutive MN elements (128 bytes) at one K index form a row, 8 rows
+// along K make a 1024-byte atom; atoms along MN are `lbo` bytes apart and
+// 8-row groups along K are `sbo` bytes apart.  A K-major tile written for one
+// product (rows = MN, 64 channels per 128-byte row) is, read this way, the
+// MN-major operand of the product that contracts over its rows.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
 // Instruction descriptor: kind::f16 with bf16 A and B (both K-major), float32
-// accumulator, shape M x N.
+// accumulator, shape M x N.  Bit 16 set makes B MN-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4)                        // D format: f32
          | (1u << 7)                      // A format: bf16

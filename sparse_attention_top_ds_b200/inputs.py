@@ -17,6 +17,11 @@ Workloads (sizes and distributions of the selection step's headline cases):
 * ``prefill``         4096 query rows x 64 heads x 128 against 32768 keys with
                       the causal prefix valid_len[t] = floor((t + c) / 4),
                       c = 4 * (S - T/4).
+* ``attention``       sparse-attention decode: 8 new tokens x 128 query heads x
+                      head_dim 512, one compressed KV cache of 32768 rows per
+                      batch row, k = 1024 selected rows drawn below a valid
+                      length ~ U{4096..32768}, a window of 128 rows, and one
+                      sink logit per head; values ~ N(0, 1).
 
 bfloat16 values are produced by drawing float32 samples and rounding them to
 the nearest bfloat16, ties to even, and are returned as uint16 bit patterns.
@@ -29,6 +34,7 @@ SEED_SAMPLING = 1002
 SEED_INDEXER = 1003
 SEED_DECODE = 1004
 SEED_PREFILL = 1005
+SEED_ATTENTION = 1006
 
 
 def rng(seed):
@@ -40,9 +46,13 @@ def f32_to_bf16_bits(x):
 
     Only finite inputs are expected (the generators draw no NaN).
     """
-    u = np.ascontiguousarray(np.asarray(x, dtype=np.float32)).view(np.uint32).astype(np.uint64)
-    bias = 0x7FFF + ((u >> 16) & 1)
-    return ((u + bias) >> 16).astype(np.uint16)
+    u = np.ascontiguousarray(np.asarray(x, dtype=np.float32)).view(np.uint32)
+    # for finite values u + 0x8000 stays below 2^32, so uint32 arithmetic is exact
+    out = (u >> np.uint32(16)) & np.uint32(1)
+    out += np.uint32(0x7FFF)
+    out += u
+    out >>= np.uint32(16)
+    return out.astype(np.uint16)
 
 
 def bf16_bits_to_f32(bits):
@@ -121,3 +131,34 @@ def sample_rows(seed, total, count):
     """A seeded, sorted subset of ``count`` distinct row indices out of ``total``."""
     g = rng(seed + 7919)
     return np.sort(g.choice(total, size=min(count, total), replace=False))
+
+
+def attention(seed=SEED_ATTENTION, batch=8, heads=128, d=512, T=32768, k=1024, W=128, shared_cache=False,
+              vl_lo=4096, vl_hi=32768, sink=True, holes=0.0, win_len=None):
+    """Sparse-attention decode inputs.
+
+    Returns a dict: q [batch, heads, d], kv [T, d] (``shared_cache``) or
+    [batch, T, d], win [batch, W, d] (bfloat16 patterns of N(0, 1) samples);
+    idx int32 [batch, k]: distinct rows drawn uniformly below a valid length
+    ~ U{vl_lo..vl_hi} (capped at T), -1 in the slots past that length; a
+    fraction ``holes`` of the slots is then replaced by -1 or by rows at or
+    past T (skipped slots); win_len int32 [batch] (given, or W); sink float32
+    [heads] ~ N(0, 1) or None.
+    """
+    g = rng(seed)
+    q = f32_to_bf16_bits(g.standard_normal((batch, heads, d), dtype=np.float32))
+    shape = (T, d) if shared_cache else (batch, T, d)
+    kv = f32_to_bf16_bits(g.standard_normal(shape, dtype=np.float32))
+    win = f32_to_bf16_bits(g.standard_normal((batch, W, d), dtype=np.float32))
+    idx = np.full((batch, k), -1, dtype=np.int32)
+    for b in range(batch):
+        L = int(min(T, g.integers(min(vl_lo, T), min(vl_hi, T), endpoint=True)))
+        m = min(k, L)
+        idx[b, :m] = g.choice(L, size=m, replace=False)
+    if holes > 0 and k > 0:
+        hit = g.random((batch, k)) < holes
+        bad = np.where(g.random((batch, k)) < 0.5, -1, T + g.integers(0, 1000, size=(batch, k)))
+        idx = np.where(hit, bad, idx).astype(np.int32)
+    wl = np.full(batch, W, dtype=np.int32) if win_len is None else np.asarray(win_len, dtype=np.int32)
+    sk = g.standard_normal(heads).astype(np.float32) if sink else None
+    return dict(q=q, kv=kv, win=win, idx=idx, win_len=wl, sink=sk)

@@ -29,8 +29,8 @@ def declared_entry_points():
 
 def test_header_declares_the_boundary():
     names = declared_entry_points()
-    for n in ("ds_topk", "ds_indexer_score", "ds_indexer_topk", "ds_get_device_status", "ds_strerror",
-              "ds_release"):
+    for n in ("ds_topk", "ds_indexer_score", "ds_indexer_topk", "ds_sparse_attention", "ds_get_device_status",
+              "ds_strerror", "ds_release"):
         assert n in names
 
 
@@ -75,6 +75,43 @@ def test_argument_errors_need_no_gpu(lib):
     assert lib.ds_indexer_topk(fake, fake, fake, 1, 65, 128, 100, None, 10, fake, None, None) == -1  # heads
     assert lib.ds_indexer_topk(fake, fake, fake, 1, 64, 128, 100, None, 0, fake, None, None) == -1   # k
     assert lib.ds_indexer_topk(fake, vp(0x100008), fake, 1, 64, 128, 100, None, 10, fake, None, None) == -1
+
+
+def test_attention_argument_errors_need_no_gpu(lib):
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    f = lib.ds_sparse_attention
+    f.restype = i32
+    f.argtypes = [vp, vp, ctypes.c_int64, i32, vp, i32, vp, i32, vp, vp, i32, i32, i32, ctypes.c_float, vp, vp, vp]
+    a = vp(0x100000)
+
+    def call(q=a, kv=a, stride=0, T=100, idx=a, k=10, win=None, W=0, wl=None, sink=None, B=2, H=128, d=512,
+             scale=0.04, out=a, lse=None):
+        return f(q, kv, stride, T, idx, k, win, W, wl, sink, B, H, d, scale, out, lse, None)
+
+    assert call(q=None) == -1
+    assert call(kv=None) == -1
+    assert call(out=None) == -1
+    assert call(d=576) == -1                  # above the largest head_dim
+    assert call(d=100) == -1                  # not a multiple of 64
+    assert call(d=0) == -1
+    assert call(T=0) == -1
+    assert call(stride=-1) == -1
+    assert call(k=2049) == -1
+    assert call(k=-1) == -1
+    assert call(idx=None) == -1               # k > 0 needs slots
+    assert call(W=8) == -1                    # a window needs rows
+    assert call(W=4097, win=a) == -1
+    assert call(B=0) == -1
+    assert call(B=65536) == -1
+    assert call(H=0) == -1
+    assert call(H=4097) == -1
+    assert call(scale=float("nan")) == -1
+    assert call(scale=float("inf")) == -1
+    assert call(q=vp(0x100008)) == -1         # 16-byte alignment
+    assert call(kv=vp(0x100004)) == -1
+    assert call(out=vp(0x100002)) == -1
+    assert call(W=8, win=vp(0x100008)) == -1
+    assert call(lse=vp(0x100002)) == -1
 
 
 def test_binding_fails_loudly_without_the_library(tmp_path):
