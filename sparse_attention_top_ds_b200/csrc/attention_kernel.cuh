@@ -9,24 +9,28 @@
 //     out[b,h,:] = sum_r e^{z_r} row_r / (sum_r e^{z_r} + e^{sink_h}),
 //     z_r = scale * (q[b,h,:] . row_r),   lse[b,h] = log of the denominator.
 //
-// How (B200 design): split-KV, one launch for the partial attentions and one
-// that combines them.
-//  * A CTA owns one batch row, a tile of 128 query heads (the M of every MMA)
-//    and a run of 64 attended slots.  The queries arrive by TMA in the
-//    128-byte-swizzled layout; the 64 rows are gathered with cp.async
-//    straight into the same layout, each row read once from HBM.
-//  * S = Q . R^T (M = 128 heads, N = 64 rows, K = d) accumulates in TMEM.
-//    Four softmax warps (one TMEM lane per head) take the chunk's maximum,
-//    write the weights 2^(z - max) as bf16 into shared memory and sum the
-//    rounded weights.
-//  * O = P . R (M = 128, N = d in pieces of at most 256, K = 64 rows) takes the
-//    gathered tile again, now as the MN-major B operand: the bytes that served
-//    as the keys serve unchanged as the values, so nothing is transposed or
-//    read twice.  O overwrites S in TMEM (the softmax has read S by then).
-//  * The epilogue stores O unnormalised with the chunk's (max, sum) in a
-//    head-fastest layout, so that every warp store is 512 contiguous bytes.
-//  * The combine kernel rescales the chunks by 2^(max_chunk - max_all), adds
-//    the sink to the normaliser, and writes out (bf16) and lse.
+// How (B200 design).  Every batch row has 128 heads that share the same rows,
+// so both products are dense: S = Q . R^T (M = heads, N = rows, K = d) and
+// O = P . R (M = heads, N = d, K = rows).  Splitting the rows over CTAs would
+// leave a float32 partial O of heads x d per CTA -- for d = 512 four times
+// the bytes of the rows themselves -- so the two products are split
+// differently, in two launches joined by programmatic dependent launch:
+//  * score kernel: a CTA owns a batch row, a tile of 128 heads and a chunk of
+//    64 attended slots.  The queries arrive by TMA (128-byte swizzle), the 64
+//    rows are gathered with cp.async straight into the same layout, S goes to
+//    TMEM, and four softmax warps (a TMEM lane per head) turn it into the
+//    chunk's weights 2^(z - max_chunk) in bf16.  The weight tile (16 KiB,
+//    already in the MMA operand layout) goes back to global memory with one
+//    bulk copy, with the chunk's (max, sum) per head.
+//  * weighted-sum kernel: a CTA owns a batch row, a tile of 128 heads and a
+//    64-column slice of d.  It reads the (max, sum) of every chunk of the row,
+//    so it knows the row's softmax maximum and normaliser, then streams the
+//    chunks through a ring: the weight tile by bulk copy, the 64-column slice
+//    of the chunk's rows by cp.async (the rows are in L2 from the score
+//    kernel).  Each weight row is rescaled in place by 2^(max_chunk - max)/sum
+//    and O_slice += P . R_slice runs on the tensor cores, the row slice being
+//    the MN-major B operand.  The accumulator is the final output: it is
+//    rounded to bf16 and written, with lse, and no combine pass is needed.
 #pragma once
 
 #include <cuda.h>
@@ -36,10 +40,12 @@
 
 namespace dstopk {
 
-constexpr int kAttnRows = 64;       // attended slots per CTA (N of S = Q . R^T)
+constexpr int kAttnRows = 64;       // attended slots per chunk (N of S = Q . R^T)
 constexpr int kAttnHeads = 128;     // query heads per CTA (M of both products)
-constexpr int kAttnThreads = 256;   // 8 warps
+constexpr int kAttnThreads = 256;   // score kernel: 8 warps
 constexpr int kAttnMaxD = 512;
+constexpr int kAttnTile = kAttnHeads * kAttnRows * 2;  // bytes of one chunk's bf16 weight tile
+constexpr int kPvSlice = 64;        // weighted-sum kernel: output columns per CTA
 
 struct AttnParams {
   const uint16_t* kv;      // bf16 compressed caches
@@ -47,30 +53,29 @@ struct AttnParams {
   const uint16_t* win;     // bf16 [B, W, D] or null
   const int32_t* idx;      // [B, k] or null
   const int32_t* win_len;  // [B] or null
-  float* opart;            // [B][HT][NS][D/4][128] float4: unnormalised O per chunk
-  float2* ml;              // [B][HT][NS][128]: (max of the chunk in log2 units, sum of weights)
+  const float* sink;       // [H] or null
+  uint8_t* ptile;          // [B][HT][NS] weight tiles of kAttnTile bytes
+  uint8_t* vtile;          // [B][D/64][NS] row tiles: the chunk's 64 rows, one 64-column block, 8 KiB
+  float2* ml;              // [B][HT][NS][128]: (chunk max in log2 units, sum of the chunk's weights)
+  uint16_t* out;           // bf16 [B, H, D]
+  float* lse;              // [B, H] or null
   int* status;
   int T, k, W, B, H, D, HT, NS;
   float scale_log2;        // scale * log2(e)
 };
 
-// Shared-memory layout for head_dim D (byte offsets from a 1024-aligned base):
-// queries D/64 blocks of 128 rows x 128 B | rows D/64 blocks of 64 x 128 B |
-// weights 128 x 128 B | row sources (64 pointers) | valid mask | 3 mbarriers |
-// TMEM slot.
-struct AttnSmem {
-  __host__ __device__ static constexpr int q_off() { return 0; }
-  __host__ __device__ static constexpr int kv_off(int D) { return (D / 64) * 16384; }
-  __host__ __device__ static constexpr int p_off(int D) { return kv_off(D) + (D / 64) * 8192; }
-  __host__ __device__ static constexpr int src_off(int D) { return p_off(D) + 16384; }
-  __host__ __device__ static constexpr int mask_off(int D) { return src_off(D) + kAttnRows * 8; }
-  __host__ __device__ static constexpr int bar_off(int D) { return mask_off(D) + 16; }
-  __host__ __device__ static constexpr int slot_off(int D) { return bar_off(D) + 32; }
-  __host__ __device__ static constexpr int bytes(int D) { return slot_off(D) + 16 + 1024; }  // + alignment slack
-};
-
-__host__ __device__ constexpr uint32_t attn_tmem_cols(int D) {
-  return D <= 64 ? 64u : (D <= 128 ? 128u : (D <= 256 ? 256u : 512u));
+// Where slot j of batch row b reads its row from; null if the slot is skipped.
+__device__ __forceinline__ const uint16_t* attn_row_src(const AttnParams& p, int b, int j) {
+  if (j < p.k) {
+    const int r = p.idx[(size_t)b * p.k + j];
+    if (r >= 0 && r < p.T) return p.kv + (long long)b * p.kv_bstride + (long long)r * p.D;
+  } else if (j < p.k + p.W) {
+    int wl = p.win_len ? p.win_len[b] : p.W;
+    wl = wl < 0 ? 0 : (wl > p.W ? p.W : wl);
+    const int i = j - p.k;
+    if (i < wl) return p.win + ((long long)b * p.W + i) * p.D;
+  }
+  return nullptr;
 }
 
 // Pack two floats into bf16x2, round to nearest even: `lo` in the low half.
@@ -80,79 +85,104 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return u;
 }
 
+// ------------------------------------------------------------------ score kernel
+
+constexpr int kRowTile = kAttnRows * 128;  // bytes of one chunk's rows in one 64-column block
+
+// Shared-memory layout for head_dim D (byte offsets from a 1024-aligned base):
+// queries D/64 blocks of 128 rows x 128 B | rows D/64 blocks of 64 x 128 B |
+// row flags (64 B) | mbarriers: queries, S | TMEM slot.
+struct AttnSmem {
+  __host__ __device__ static constexpr int q_off() { return 0; }
+  __host__ __device__ static constexpr int kv_off(int D) { return (D / 64) * 16384; }
+  __host__ __device__ static constexpr int flag_off(int D) { return kv_off(D) + (D / 64) * kRowTile; }
+  __host__ __device__ static constexpr int bar_off(int D) { return flag_off(D) + kAttnRows; }
+  __host__ __device__ static constexpr int slot_off(int D) { return bar_off(D) + 16; }
+  __host__ __device__ static constexpr int bytes(int D) { return slot_off(D) + 16 + 1024; }  // + alignment slack
+};
+
+// tm_q views the queries [rows][D] as (64 channels, rows, D/64 blocks), so one
+// box of (64, 128, D/64) lands in shared memory block by block, each block
+// 128 rows x 128 B in the 128-byte-swizzled layout.
 __global__ void __launch_bounds__(kAttnThreads, 1)
-    sparse_attn_partial_kernel(const __grid_constant__ CUtensorMap tm_q, const AttnParams p) {
+    sparse_attn_score_kernel(const __grid_constant__ CUtensorMap tm_q, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const int D = p.D, DB = D >> 6;
   const uint32_t q_s = sbase + AttnSmem::q_off();
   const uint32_t kv_s = sbase + AttnSmem::kv_off(D);
-  const uint32_t p_s = sbase + AttnSmem::p_off(D);
-  const uint16_t** src = reinterpret_cast<const uint16_t**>(smem + AttnSmem::src_off(D));
-  uint32_t* mask = reinterpret_cast<uint32_t*>(smem + AttnSmem::mask_off(D));
+  uint8_t* flags = smem + AttnSmem::flag_off(D);
   const uint32_t bar_q = sbase + AttnSmem::bar_off(D);
-  const uint32_t bar_s = bar_q + 8, bar_o = bar_q + 16;
+  const uint32_t bar_s = bar_q + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + AttnSmem::slot_off(D));
 
   const int split = blockIdx.x, ht = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t ncols = attn_tmem_cols(D);
+  constexpr uint32_t kCols = 64;
 
   if (tid == 0) {
     mbar_init(bar_q, 1);
     mbar_init(bar_s, 1);
-    mbar_init(bar_o, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), ncols);
+    tmem_alloc(smem_u32(tmem_slot), kCols);
     tmem_relinquish();
   }
-  // the slots (and the queries) may be written by the kernel just before this one
-  pdl_wait();
-  if (tid == 0) {
-    tma_prefetch_desc(&tm_q);
-    mbar_arrive_expect_tx(bar_q, (uint32_t)DB * 16384u);
-    for (int db = 0; db < DB; ++db)
-      tma_load_2d(q_s + (uint32_t)db * 16384u, &tm_q, db * 64, b * p.H + ht * kAttnHeads, bar_q);
-  }
-  // where each of the 64 slots reads its row from (null: skipped)
-  if (tid < kAttnRows) {
-    const int j = split * kAttnRows + tid;
-    const uint16_t* s = nullptr;
-    if (j < p.k) {
-      const int r = p.idx[(size_t)b * p.k + j];
-      if (r >= 0 && r < p.T) s = p.kv + (long long)b * p.kv_bstride + (long long)r * D;
-    } else if (j < p.k + p.W) {
-      int wl = p.win_len ? p.win_len[b] : p.W;
-      wl = wl < 0 ? 0 : (wl > p.W ? p.W : wl);
-      const int i = j - p.k;
-      if (i < wl) s = p.win + ((long long)b * p.W + i) * D;
-    }
-    src[tid] = s;
-    const uint32_t bal = __ballot_sync(0xffffffffu, s != nullptr);
-    if (lane == 0) mask[warp] = bal;
-  }
-  __syncthreads();
-
-  // gather: 16-byte pieces into the swizzled layout (piece c8 of row r goes to
-  // position c8 ^ (r & 7) of the row's 128 bytes); skipped rows become zeros
-  for (int c = tid; c < DB * 512; c += kAttnThreads) {
-    const int db = c >> 9, rem = c & 511, r = rem >> 3, c8 = rem & 7;
-    const uint16_t* s = src[r];
-    const uint32_t dst = kv_s + (uint32_t)db * 8192u + (uint32_t)r * 128u + ((uint32_t)(c8 ^ (r & 7)) << 4);
-    const void* g = s ? static_cast<const void*>(s + db * 64 + c8 * 8) : static_cast<const void*>(p.kv);
-    const uint32_t nbytes = s ? 16u : 0u;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(g), "r"(nbytes) : "memory");
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the slots (and the queries) may be written by the kernel just before this one
+  pdl_wait();
+  // let the weighted-sum kernel launch now: its CTAs take SMs as these exit,
+  // and wait (griddepcontrol.wait) for this whole grid before reading
+  pdl_launch_dependents();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_q, (uint32_t)DB * 16384u);
+    tma_load_3d(q_s, &tm_q, 0, b * p.H + ht * kAttnHeads, 0, bar_q);
+  }
+  // gather: thread t moves 16-byte piece c8 = t % 8 of rows t / 8 and t / 8 + 32
+  // of every 64-column block, all loads in flight at once, into the swizzled
+  // layout (piece c8 of row r goes to position c8 ^ (r & 7) of the row's 128
+  // bytes); skipped rows become zeros.  The first head tile also stores each
+  // block's row tile for the weighted-sum kernel.
+  {
+    const int r0 = tid >> 3, r1 = r0 + 32, c8 = tid & 7;
+    const uint16_t* s0 = attn_row_src(p, b, split * kAttnRows + r0);
+    const uint16_t* s1 = attn_row_src(p, b, split * kAttnRows + r1);
+    if (c8 == 0) {
+      flags[r0] = s0 != nullptr;
+      flags[r1] = s1 != nullptr;
+    }
+    uint4 v0[kAttnMaxD / 64], v1[kAttnMaxD / 64];
+#pragma unroll
+    for (int db = 0; db < kAttnMaxD / 64; ++db) {
+      if (db < DB) {
+        v0[db] = s0 ? __ldcg(reinterpret_cast<const uint4*>(s0 + db * 64 + c8 * 8)) : make_uint4(0, 0, 0, 0);
+        v1[db] = s1 ? __ldcg(reinterpret_cast<const uint4*>(s1 + db * 64 + c8 * 8)) : make_uint4(0, 0, 0, 0);
+      }
+    }
+    const uint32_t o0 = (uint32_t)r0 * 128u + ((uint32_t)(c8 ^ (r0 & 7)) << 4);
+    const uint32_t o1 = (uint32_t)r1 * 128u + ((uint32_t)(c8 ^ (r1 & 7)) << 4);
+    uint8_t* vt = (ht == 0) ? p.vtile + ((size_t)b * DB * p.NS + split) * kRowTile : nullptr;
+#pragma unroll
+    for (int db = 0; db < kAttnMaxD / 64; ++db) {
+      if (db < DB) {
+        sts128(kv_s + (uint32_t)db * kRowTile + o0, v0[db]);
+        sts128(kv_s + (uint32_t)db * kRowTile + o1, v1[db]);
+        if (vt) {
+          uint8_t* t = vt + (size_t)db * p.NS * kRowTile;
+          *reinterpret_cast<uint4*>(t + o0) = v0[db];
+          *reinterpret_cast<uint4*>(t + o1) = v1[db];
+        }
+      }
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
 
   // ---- S = Q . R^T into TMEM columns [0, 64)
   if (tid == 0) {
@@ -164,7 +194,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t a = sw128_kmajor_desc(q_s + (uint32_t)db * 16384u + (uint32_t)kk * 32u);
-          const uint64_t bd = sw128_kmajor_desc(kv_s + (uint32_t)db * 8192u + (uint32_t)kk * 32u);
+          const uint64_t bd = sw128_kmajor_desc(kv_s + (uint32_t)db * kRowTile + (uint32_t)kk * 32u);
           mma_bf16_ss(tmem, a, bd, idesc, (db | kk) != 0 ? 1u : 0u);
         }
       }
@@ -172,157 +202,297 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mma_commit(bar_s);  // arrives even when nothing was issued, so that no one waits for ever
   }
 
-  // ---- softmax of the chunk: warps 0..3, TMEM lane = head
-  float m_row = -INFINITY, l_row = 0.0f;
-  if (warp < 4) {
+  // ---- the chunk's weights: all 8 warps, TMEM lane = head (lane quarter =
+  // warp % 4), warps 0..3 taking rows 0..31 of the chunk and warps 4..7 rows
+  // 32..63; the two halves of a head swap their maxima and sums through shared
+  // memory.  Each thread writes its half of the head's 128-byte row of the
+  // tile straight to global memory, in the swizzled order the weighted-sum
+  // kernel's MMAs read.
+  const size_t chunk = ((size_t)b * p.HT + ht) * p.NS + split;
+  {
+    const int half = warp >> 2;
+    const int h = (warp & 3) * 32 + lane;
+    float* xch = reinterpret_cast<float*>(smem + AttnSmem::kv_off(D));  // the row tiles are no longer read
     mbar_wait_bounded(bar_s, 0, p.status);
     __syncwarp();
     tc_fence_after();
-    const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
-    uint32_t r[64];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) tmem_ld16(taddr + (uint32_t)(c * 16), *reinterpret_cast<uint32_t(*)[16]>(r + c * 16));
+    const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(half * 32);
+    uint32_t r[32];
+    tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
+    tmem_ld16(taddr + 16u, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+    const uint4 fa = *reinterpret_cast<const uint4*>(flags + half * 32);
+    const uint4 fb = *reinterpret_cast<const uint4*>(flags + half * 32 + 16);
+    const uint32_t fw[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
     tmem_wait_ld();
-    const uint32_t m0 = mask[0], m1 = mask[1];
-    float z[64];
+    float z[32];
+    float m = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < 64; ++j) {
-      const bool v = ((j < 32 ? m0 >> j : m1 >> (j - 32)) & 1u) != 0;
+    for (int j = 0; j < 32; ++j) {
+      const bool v = ((fw[j >> 2] >> ((j & 3) * 8)) & 0xffu) != 0;
       z[j] = v ? __uint_as_float(r[j]) * p.scale_log2 : -INFINITY;
-      m_row = fmaxf(m_row, z[j]);
+      m = fmaxf(m, z[j]);
     }
-    const int h = warp * 32 + lane;
-    const uint32_t prow = p_s + (uint32_t)h * 128u;
+    xch[half * kAttnHeads + h] = m;
+    named_bar_sync(1, kAttnThreads);
+    m = fmaxf(m, xch[(1 - half) * kAttnHeads + h]);
+    const float mu = m == -INFINITY ? 0.0f : m;  // exp2(-inf - mu) = 0 for every skipped row
+    float l = 0.0f;
+    uint4* trow = reinterpret_cast<uint4*>(p.ptile + chunk * (size_t)kAttnTile + (size_t)h * 128u);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < 4; ++c) {
       uint32_t pk[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int j = c * 8 + i * 2;
-        const float e0 = z[j] == -INFINITY ? 0.0f : exp2f(z[j] - m_row);
-        const float e1 = z[j + 1] == -INFINITY ? 0.0f : exp2f(z[j + 1] - m_row);
-        const uint32_t u = pack_bf16x2(e0, e1);
-        l_row += __uint_as_float(u << 16) + __uint_as_float(u & 0xffff0000u);
+        const uint32_t u = pack_bf16x2(exp2f(z[j] - mu), exp2f(z[j + 1] - mu));
+        l += __uint_as_float(u << 16) + __uint_as_float(u & 0xffff0000u);
         pk[i] = u;
       }
-      sts128(prow + ((uint32_t)(c ^ (h & 7)) << 4), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+      trow[(half * 4 + c) ^ (h & 7)] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
+    xch[2 * kAttnHeads + half * kAttnHeads + h] = l;
+    named_bar_sync(1, kAttnThreads);
+    if (half == 0) p.ml[chunk * kAttnHeads + h] = make_float2(m, l + xch[3 * kAttnHeads + h]);
   }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-
-  // ---- O = P . R: the gathered tile again, as the MN-major B operand
-  if (tid == 0) {
-    tc_fence_after();
-    for (int n0 = 0; n0 < D; n0 += 256) {
-      const int N = D - n0 < 256 ? D - n0 : 256;
-      const uint32_t idesc = idesc_bf16_f32(128, N) | (1u << 16);  // B is MN-major
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t a = sw128_kmajor_desc(p_s + (uint32_t)kk * 32u);
-        const uint64_t bd =
-            sw128_mnmajor_desc(kv_s + (uint32_t)(n0 / 64) * 8192u + (uint32_t)kk * 2048u, 8192u, 1024u);
-        mma_bf16_ss(tmem + (uint32_t)n0, a, bd, idesc, kk > 0 ? 1u : 0u);
-      }
-    }
-    mma_commit(bar_o);
-  }
-
-  // ---- epilogue: 8 warps, TMEM lane quarter = warp % 4, column half = warp / 4
-  mbar_wait_bounded(bar_o, 0, p.status);
-  __syncwarp();
-  tc_fence_after();
-  {
-    const int qd = warp & 3, half = warp >> 2;
-    const int hrow = qd * 32 + lane;
-    const uint32_t taddr = tmem + ((uint32_t)(qd * 32) << 16);
-    const size_t chunk = ((size_t)b * p.HT + ht) * p.NS + split;
-    float4* op = reinterpret_cast<float4*>(p.opart) + chunk * (size_t)(D / 4) * kAttnHeads + hrow;
-    const int c_lo = half * (D / 2), c_hi = c_lo + D / 2;
-    for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
-      uint32_t r[32];
-      tmem_ld16(taddr + (uint32_t)c0, *reinterpret_cast<uint32_t(*)[16]>(r));
-      tmem_ld16(taddr + (uint32_t)(c0 + 16), *reinterpret_cast<uint32_t(*)[16]>(r + 16));
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        op[(size_t)(c0 / 4 + i) * kAttnHeads] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                                            __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-    }
-    if (warp < 4) p.ml[chunk * kAttnHeads + hrow] = make_float2(m_row, l_row);
-  }
-
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, ncols);
+    tmem_dealloc(tmem, kCols);
   }
-  pdl_launch_dependents();
 }
 
-// ------------------------------------------------------------------ combine
+// ------------------------------------------------------------------ weighted-sum kernel
 
-struct AttnCombineParams {
-  const float* opart;
-  const float2* ml;
-  const float* sink;   // [H] or null
-  uint16_t* out;       // bf16 [B, H, D]
-  float* lse;          // [B, H] or null
-  int B, H, D, HT, NS;
+// Warp roles: lane 0 of warp 0 loads; warps 1..8 rescale the weight rows (two
+// threads per head, half a row each) and later read the accumulator; warp 9
+// owns TMEM and issues the MMAs from one thread.  A ring stage holds K
+// consecutive chunks: their weight tiles (K x 16 KiB) and their row tiles for
+// this CTA's 64 columns (K x 8 KiB), each a contiguous run in global memory
+// fetched by one bulk copy (large copies keep the copy engine near its peak).
+// Stages pass full -> ready -> empty through mbarriers, so no CTA-wide
+// barrier sits in the loop.
+//
+// With G = 2 the chunks of a batch row are split between the two CTAs of a
+// cluster.  Both know the row's softmax maximum and normaliser, so their two
+// accumulators are partial sums of the same normalised output: each CTA sends
+// the partner the 32 columns the partner finalises, by st.async into the
+// partner's shared memory completing on the partner's mbarrier, and each
+// writes 32 columns.
+constexpr int kPvWarps = 10;
+constexpr int kPvRescale = 256;  // rescaling threads (warps 1..8)
+constexpr int kPvStages = 2;
+template <int K>
+struct PvSmem {
+  static constexpr int kStage = K * (kAttnTile + kRowTile);
+  // ring | partner's columns (128 heads x 32 floats) | (max, sum) of every chunk
+  // of the row | mbarriers full[2], ready[2], empty[2], ml, done, recv | TMEM slot
+  __host__ __device__ static constexpr int recv_off() { return kPvStages * kStage; }
+  __host__ __device__ static constexpr int ml_off() { return recv_off() + kAttnHeads * 32 * 4; }
+  __host__ __device__ static constexpr int bar_off(int NS) { return ml_off() + NS * kAttnHeads * 8; }
+  __host__ __device__ static constexpr int slot_off(int NS) { return bar_off(NS) + (3 * kPvStages + 3) * 8; }
+  __host__ __device__ static constexpr int bytes(int NS) { return slot_off(NS) + 16 + 1024; }
 };
 
-// Grid (D/64 column blocks, ceil(H/32) head groups, B); 4 warps.  Lane = head,
-// warp w covers 16 columns, so every load of a chunk's O is 512 contiguous
-// bytes.
-__global__ void __launch_bounds__(128) sparse_attn_combine_kernel(const AttnCombineParams p) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cb = blockIdx.x, b = blockIdx.z;
-  const int h = blockIdx.y * 32 + lane;
-  pdl_wait();
-  if (h >= p.H) return;
+// Columns [LO, LO + 32) of one head's accumulator, held as r[0..31]:
+// optionally add the partner's share from `recv`, round to bf16 and store.
+template <bool ADD>
+__device__ __forceinline__ void pv_emit(const uint32_t (&r)[32], const float* recv, uint16_t* dst) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * q + e]) + (ADD ? recv[8 * q + e] : 0.0f);
+    d4[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                       pack_bf16x2(v[6], v[7]));
+  }
+}
+
+template <int K>
+__global__ void __launch_bounds__(kPvWarps * 32, 1) sparse_attn_pv_kernel(const AttnParams p) {
+  using L_ = PvSmem<K>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int NS = p.NS;
+  const int G = gridDim.y, g = blockIdx.y;  // chunk group = rank in the cluster
+  const int NSg = (NS + G - 1) / G;
+  const int c0 = g * NSg, nmine = max(0, min(NS, c0 + NSg) - c0);
+  const int nstage = (nmine + K - 1) / K;   // ring uses of this CTA
+  const float2* ml_s = reinterpret_cast<const float2*>(smem + L_::ml_off());
+  float* recv = reinterpret_cast<float*>(smem + L_::recv_off());
+  const uint32_t full0 = sbase + L_::bar_off(NS);
+  const uint32_t ready0 = full0 + 8u * kPvStages, empty0 = ready0 + 8u * kPvStages;
+  const uint32_t bar_ml = empty0 + 8u * kPvStages, bar_done = bar_ml + 8u, bar_recv = bar_done + 8u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L_::slot_off(NS));
+  const int slice = blockIdx.x, ht = blockIdx.z % p.HT, b = blockIdx.z / p.HT;
+  const int DB = p.D >> 6;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr uint32_t kCols = kPvSlice;
   constexpr float kLog2e = 1.4426950408889634f;
   constexpr float kLn2 = 0.6931471805599453f;
-  const int ht = h / kAttnHeads, hl = h % kAttnHeads;
-  const size_t base = ((size_t)b * p.HT + ht) * p.NS;
-  const float2* ml = p.ml + base * kAttnHeads + hl;
-  const float sink_l2 = p.sink ? p.sink[h] * kLog2e : -INFINITY;
-  float M = sink_l2;
-  for (int s = 0; s < p.NS; ++s) {
-    const float2 v = ml[(size_t)s * kAttnHeads];
-    if (v.y > 0.0f) M = fmaxf(M, v.x);
+
+  if (tid == 0) {
+    for (int s = 0; s < kPvStages; ++s) {
+      mbar_init(full0 + 8u * s, 1);             // the producer's expect_tx
+      mbar_init(ready0 + 8u * s, kPvRescale);   // the rescaling threads
+      mbar_init(empty0 + 8u * s, 1);            // the MMAs' commit
+    }
+    mbar_init(bar_ml, 1);
+    mbar_init(bar_done, 1);
+    mbar_init(bar_recv, 1);
+    fence_mbar_init();
   }
-  float L = p.sink ? exp2f(sink_l2 - M) : 0.0f;
-  float acc[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
-  const int cc0 = cb * 16 + warp * 4;  // first float4 column of this warp
-  const float4* op = reinterpret_cast<const float4*>(p.opart) + base * (size_t)(p.D / 4) * kAttnHeads + hl;
-  for (int s = 0; s < p.NS; ++s) {
-    const float2 v = ml[(size_t)s * kAttnHeads];
-    if (v.y > 0.0f) {
-      const float w = exp2f(v.x - M);
-      L = fmaf(w, v.y, L);
-      const float4* o = op + (size_t)s * (p.D / 4) * kAttnHeads;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 x = o[(size_t)(cc0 + i) * kAttnHeads];
-        acc[4 * i] = fmaf(w, x.x, acc[4 * i]);
-        acc[4 * i + 1] = fmaf(w, x.y, acc[4 * i + 1]);
-        acc[4 * i + 2] = fmaf(w, x.z, acc[4 * i + 2]);
-        acc[4 * i + 3] = fmaf(w, x.w, acc[4 * i + 3]);
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (G == 2) cluster_sync();  // the partner's mbarriers exist before anything targets them
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // the tiles and statistics come from the score kernel
+
+  const size_t row0 = ((size_t)b * p.HT + ht) * NS;          // this row's first weight tile
+  const size_t vrow0 = ((size_t)b * DB + slice) * NS;         // this row's first row tile of this slice
+  float M = -INFINITY, L = 0.0f;  // head h's softmax maximum and normaliser (warps 1..8)
+  // warps 1..8 own half a head row per thread; a warp may only read its TMEM
+  // lane quarter (warp % 4), so warp w takes heads 32 (w % 4) .. + 31, and
+  // warps 1..4 the first half of each row, warps 5..8 the second
+  const int h = ((warp & 3) << 5) | lane;
+  const int half = (warp - 1) >> 2;
+  if (warp == 0) {
+    // ---------------- producer
+    if (lane == 0) {
+      if (NS > 0) {
+        const uint32_t bytes = (uint32_t)NS * kAttnHeads * 8u;
+        mbar_arrive_expect_tx(bar_ml, bytes);
+        bulk_g2s(sbase + L_::ml_off(), p.ml + row0 * kAttnHeads, bytes, bar_ml);
+      }
+      for (int j = 0; j < nstage; ++j) {
+        const int s = j % kPvStages;
+        const int c = c0 + j * K, n = min(K, c0 + nmine - c);
+        if (j >= kPvStages) mbar_wait_bounded(empty0 + 8u * s, (uint32_t)((j / kPvStages - 1) & 1), p.status);
+        const uint32_t st = sbase + (uint32_t)s * L_::kStage;
+        mbar_arrive_expect_tx(full0 + 8u * s, (uint32_t)n * (kAttnTile + kRowTile));
+        bulk_g2s(st, p.ptile + (row0 + c) * (size_t)kAttnTile, (uint32_t)n * kAttnTile, full0 + 8u * s);
+        bulk_g2s(st + (uint32_t)K * kAttnTile, p.vtile + (vrow0 + c) * (size_t)kRowTile, (uint32_t)n * kRowTile,
+                 full0 + 8u * s);
       }
     }
-  }
-  const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-  uint32_t pk[8];
+  } else if (warp <= 8) {
+    // ---------------- rescaling: head h's weights of every chunk, to the row's
+    // maximum and normaliser.  Every 16-byte piece of a row takes the same
+    // factor, so the thread visits its pieces in the order q ^ (h % 8): eight
+    // consecutive heads then touch eight different bank groups.
+    const int hg = ht * kAttnHeads + h;
+    const float sink_l2 = (p.sink && hg < p.H) ? p.sink[hg] * kLog2e : -INFINITY;
+    M = sink_l2;
+    if (NS > 0) mbar_wait_bounded(bar_ml, 0, p.status);
+    for (int c = 0; c < NS; ++c) {
+      const float2 v = ml_s[c * kAttnHeads + h];
+      if (v.y > 0.0f) M = fmaxf(M, v.x);
+    }
+    if (M > -INFINITY && sink_l2 > -INFINITY) L = exp2f(sink_l2 - M);
+    for (int c = 0; c < NS; ++c) {
+      const float2 v = ml_s[c * kAttnHeads + h];
+      if (v.y > 0.0f) L = fmaf(v.y, exp2f(v.x - M), L);
+    }
+    const float invL = L > 0.0f ? 1.0f / L : 0.0f;
+    for (int j = 0; j < nstage; ++j) {
+      const int s = j % kPvStages;
+      const int c = c0 + j * K, n = min(K, c0 + nmine - c);
+      mbar_wait_bounded(full0 + 8u * s, (uint32_t)((j / kPvStages) & 1), p.status);
+      for (int t = 0; t < n; ++t) {
+        const float2 v = ml_s[(c + t) * kAttnHeads + h];
+        const float f = v.y > 0.0f ? exp2f(v.x - M) * invL : 0.0f;
+        const uint32_t prow = sbase + (uint32_t)s * L_::kStage + (uint32_t)t * kAttnTile + (uint32_t)h * 128u;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(acc[2 * i] * inv, acc[2 * i + 1] * inv);
-  uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)b * p.H + h) * p.D + (size_t)cc0 * 4);
-  dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-  if (cb == 0 && warp == 0 && p.lse) p.lse[(size_t)b * p.H + h] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t a = prow + ((uint32_t)((half * 4 + q) ^ (h & 7)) << 4);
+          uint4 x = lds128(a);
+          uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(w[e] << 16) * f, __uint_as_float(w[e] & 0xffff0000u) * f);
+          sts128(a, x);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(ready0 + 8u * s);
+    }
+  } else if (lane == 0) {
+    // ---------------- MMA issuer: O_slice += P'_chunk . R_slice
+    constexpr uint32_t idesc = idesc_bf16_f32(128, kPvSlice) | (1u << 16);  // B is MN-major
+    for (int j = 0; j < nstage; ++j) {
+      const int s = j % kPvStages;
+      const int n = min(K, c0 + nmine - (c0 + j * K));
+      mbar_wait_bounded(ready0 + 8u * s, (uint32_t)((j / kPvStages) & 1), p.status);
+      fence_proxy_async_smem();
+      tc_fence_after();
+      const uint32_t st = sbase + (uint32_t)s * L_::kStage;
+      for (int t = 0; t < n; ++t) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t a = sw128_kmajor_desc(st + (uint32_t)t * kAttnTile + (uint32_t)kk * 32u);
+          const uint64_t bd = sw128_mnmajor_desc(st + (uint32_t)K * kAttnTile + (uint32_t)t * kRowTile +
+                                                     (uint32_t)kk * 2048u, 8192u, 1024u);
+          mma_bf16_ss(tmem, a, bd, idesc, (j | t | kk) != 0 ? 1u : 0u);
+        }
+      }
+      mma_commit(empty0 + 8u * s);
+    }
+    mma_commit(bar_done);  // after every MMA above (or at once if there were none)
+  }
+
+  // ---- epilogue: warps 1..8, thread (h, half) holds columns [32 half, 32 half + 32)
+  if (warp >= 1 && warp <= 8) {
+    uint32_t r[32];
+    if (nmine > 0) {
+      mbar_wait_bounded(bar_done, 0, p.status);
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(half * 32);
+      tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
+      tmem_ld16(taddr + 16u, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) r[i] = 0u;
+    }
+    const int hg = ht * kAttnHeads + h;
+    uint16_t* orow = p.out + ((size_t)b * p.H + hg) * p.D + (size_t)slice * kPvSlice + half * 32;
+    if (G == 2) {
+      if (half != g) {
+        // these 32 columns are finalised by the partner (CTA `half` of the pair)
+        const uint32_t dst = dsmem_map(smem_u32(recv + h * 32), (uint32_t)half);
+        const uint32_t rbar = dsmem_map(bar_recv, (uint32_t)half);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::
+                           "r"(dst + 16u * q), "r"(r[4 * q]), "r"(r[4 * q + 1]), "r"(r[4 * q + 2]), "r"(r[4 * q + 3]),
+                       "r"(rbar)
+                       : "memory");
+      } else {
+        if (h == 0) mbar_arrive_expect_tx(bar_recv, kAttnHeads * 32 * 4);  // 128 heads x 32 columns from the partner
+        mbar_wait_bounded(bar_recv, 0, p.status);
+        if (hg < p.H) pv_emit<true>(r, recv + h * 32, orow);
+      }
+    } else if (hg < p.H) {
+      pv_emit<false>(r, recv, orow);
+    }
+    if (half == 0 && hg < p.H && slice == 0 && g == 0 && p.lse)
+      p.lse[(size_t)b * p.H + hg] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCols);
+  }
+  pdl_launch_dependents();
 }
 
 }  // namespace dstopk

@@ -316,8 +316,16 @@ static cudaError_t indexer_setup() {
     e = cudaFuncSetAttribute(indexer_topk_rowcluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              RcSmem::kBytes);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(sparse_attn_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(sparse_attn_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnSmem::bytes(kAttnMaxD));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(sparse_attn_pv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(sparse_attn_pv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(sparse_attn_pv_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(sparse_attn_pv_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   return e;
 }
 
@@ -580,13 +588,14 @@ static void* get_scratch(DeviceState* s, size_t bytes) {
 
 // ---- sparse attention over the selected rows
 
-// Queries [rows][D] bf16 in boxes of 64 channels x 128 heads, 128-byte swizzle.
+// Queries [rows][D] bf16 viewed as (64 channels, rows, D/64 blocks): one box
+// of (64, 128, D/64) is a head tile's queries, block by block, 128-byte swizzle.
 static bool encode_attn_q(const void* q, long long rows, int D, CUtensorMap* tq) {
-  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-  cuuint64_t str[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)kAttnHeads};
-  cuuint32_t one[2] = {1, 1};
-  const CUresult r = g_encode(tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, str, box, one,
+  cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(D / 64)};
+  cuuint64_t str[2] = {(cuuint64_t)D * 2, 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)kAttnHeads, (cuuint32_t)(D / 64)};
+  cuuint32_t one[3] = {1, 1, 1};
+  const CUresult r = g_encode(tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, str, box, one,
                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -617,76 +626,97 @@ static int attention_enqueue(const uint16_t* q, const uint16_t* kv, long long kv
                              cudaStream_t st, DeviceState* s) {
   const int HT = (H + kAttnHeads - 1) / kAttnHeads;
   const int NS = (k + W + kAttnRows - 1) / kAttnRows;
-  const size_t opart_row = (size_t)HT * NS * (size_t)D * kAttnHeads * sizeof(float);
+  // per batch row and chunk: a bf16 weight tile and (max, sum) per head of
+  // every head tile, and the chunk's rows as D/64 row tiles
+  const size_t tile_row = (size_t)HT * NS * kAttnTile;
+  const size_t vt_row = (size_t)(D / 64) * NS * kRowTile;
   const size_t ml_row = (size_t)HT * NS * kAttnHeads * sizeof(float2);
+  const size_t per_row = tile_row + vt_row + ml_row;
   int per = B;
-  if (NS > 0 && (opart_row + ml_row) * (size_t)B > kAttnScratchCap)
-    per = (int)std::max<size_t>(1, kAttnScratchCap / (opart_row + ml_row));
-  float* opart = nullptr;
+  if (NS > 0 && per_row * (size_t)B > kAttnScratchCap) per = (int)std::max<size_t>(1, kAttnScratchCap / per_row);
+  uint8_t* ptile = nullptr;
+  uint8_t* vtile = nullptr;
   float2* ml = nullptr;
   if (NS > 0) {
-    uint8_t* base = static_cast<uint8_t*>(get_attn_scratch(s, (opart_row + ml_row) * (size_t)per));
+    uint8_t* base = static_cast<uint8_t*>(get_attn_scratch(s, per_row * (size_t)per));
     if (!base) return DS_ERR_NOMEM;
-    opart = reinterpret_cast<float*>(base);
-    ml = reinterpret_cast<float2*>(base + opart_row * (size_t)per);
+    ptile = base;
+    vtile = base + tile_row * (size_t)per;
+    ml = reinterpret_cast<float2*>(vtile + vt_row * (size_t)per);
   }
   const float kLog2e = 1.4426950408889634f;
   for (int b0 = 0; b0 < B; b0 += per) {
     const int nb = std::min(per, B - b0);
+    AttnParams p;
+    p.kv = kv + (size_t)b0 * (size_t)kv_bstride_rows * D;
+    p.kv_bstride = kv_bstride_rows * (long long)D;
+    p.win = win ? win + (size_t)b0 * W * D : nullptr;
+    p.idx = idx ? idx + (size_t)b0 * k : nullptr;
+    p.win_len = win_len ? win_len + b0 : nullptr;
+    p.sink = sink;
+    p.ptile = ptile;
+    p.vtile = vtile;
+    p.ml = ml;
+    p.out = out + (size_t)b0 * H * D;
+    p.lse = lse ? lse + (size_t)b0 * H : nullptr;
+    p.status = s->status;
+    p.T = T;
+    p.k = k;
+    p.W = W;
+    p.B = nb;
+    p.H = H;
+    p.D = D;
+    p.HT = HT;
+    p.NS = NS;
+    p.scale_log2 = scale * kLog2e;
+    cudaLaunchAttribute attr[1];
+    set_pdl(attr[0]);
     if (NS > 0) {
       CUtensorMap tq;
       if (!encode_attn_q(q + (size_t)b0 * H * D, (long long)nb * H, D, &tq)) return DS_ERR_ARG;
-      AttnParams p;
-      p.kv = kv + (size_t)b0 * (size_t)kv_bstride_rows * D;
-      p.kv_bstride = kv_bstride_rows * (long long)D;
-      p.win = win ? win + (size_t)b0 * W * D : nullptr;
-      p.idx = idx ? idx + (size_t)b0 * k : nullptr;
-      p.win_len = win_len ? win_len + b0 : nullptr;
-      p.opart = opart;
-      p.ml = ml;
-      p.status = s->status;
-      p.T = T;
-      p.k = k;
-      p.W = W;
-      p.B = nb;
-      p.H = H;
-      p.D = D;
-      p.HT = HT;
-      p.NS = NS;
-      p.scale_log2 = scale * kLog2e;
       cudaLaunchConfig_t cfg;
       memset(&cfg, 0, sizeof(cfg));
       cfg.gridDim = dim3((unsigned)NS, (unsigned)HT, (unsigned)nb);
       cfg.blockDim = dim3(kAttnThreads, 1, 1);
       cfg.dynamicSmemBytes = (size_t)AttnSmem::bytes(D);
       cfg.stream = st;
-      cudaLaunchAttribute attr[1];
-      set_pdl(attr[0]);
       cfg.attrs = attr;
       cfg.numAttrs = pdl_on() ? 1 : 0;
-      if (cudaLaunchKernelEx(&cfg, sparse_attn_partial_kernel, tq, p) != cudaSuccess) return DS_ERR_CUDA;
+      if (cudaLaunchKernelEx(&cfg, sparse_attn_score_kernel, tq, p) != cudaSuccess) return DS_ERR_CUDA;
     }
-    AttnCombineParams c;
-    c.opart = opart;
-    c.ml = ml;
-    c.sink = sink;
-    c.out = out + (size_t)b0 * H * D;
-    c.lse = lse ? lse + (size_t)b0 * H : nullptr;
-    c.B = nb;
-    c.H = H;
-    c.D = D;
-    c.HT = HT;
-    c.NS = NS;
+    // chunks of a row split over a cluster pair while one CTA per column slice
+    // would leave more than half of the SMs idle
+    const int G = (NS > 1 && 2L * (D / kPvSlice) * HT * nb <= s->num_sms) ? 2 : 1;
+    // the most chunks per ring stage that the row's statistics leave room for
+    const int lim = 227 * 1024;
+    const int K = PvSmem<4>::bytes(NS) <= lim ? 4 : (PvSmem<3>::bytes(NS) <= lim ? 3 : (PvSmem<2>::bytes(NS) <= lim ? 2 : 1));
+    if (PvSmem<1>::bytes(NS) > lim) return DS_ERR_ARG;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3((unsigned)(D / 64), (unsigned)((H + 31) / 32), (unsigned)nb);
-    cfg.blockDim = dim3(128, 1, 1);
+    cfg.gridDim = dim3((unsigned)(D / kPvSlice), (unsigned)G, (unsigned)(HT * nb));
+    cfg.blockDim = dim3(kPvWarps * 32, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)(K == 4   ? PvSmem<4>::bytes(NS)
+                                    : K == 3 ? PvSmem<3>::bytes(NS)
+                                    : K == 2 ? PvSmem<2>::bytes(NS)
+                                             : PvSmem<1>::bytes(NS));
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    set_pdl(attr[0]);
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl_on() ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, sparse_attn_combine_kernel, c) != cudaSuccess) return DS_ERR_CUDA;
+    cudaLaunchAttribute pattr[2];
+    int na = 0;
+    if (pdl_on()) set_pdl(pattr[na++]);
+    if (G == 2) {
+      pattr[na].id = cudaLaunchAttributeClusterDimension;
+      pattr[na].val.clusterDim.x = 1;
+      pattr[na].val.clusterDim.y = 2;
+      pattr[na].val.clusterDim.z = 1;
+      ++na;
+    }
+    cfg.attrs = pattr;
+    cfg.numAttrs = na;
+    const cudaError_t e = K == 4   ? cudaLaunchKernelEx(&cfg, sparse_attn_pv_kernel<4>, p)
+                          : K == 3 ? cudaLaunchKernelEx(&cfg, sparse_attn_pv_kernel<3>, p)
+                          : K == 2 ? cudaLaunchKernelEx(&cfg, sparse_attn_pv_kernel<2>, p)
+                                   : cudaLaunchKernelEx(&cfg, sparse_attn_pv_kernel<1>, p);
+    if (e != cudaSuccess) return DS_ERR_CUDA;
   }
   return DS_OK;
 }
@@ -851,6 +881,7 @@ extern "C" int ds_sparse_attention(const void* q, const void* kv, int64_t kv_bat
                                    int batch, int heads, int d, float scale, void* out, float* lse, void* stream) {
   auto misaligned = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; };
   if (!q || !kv || !out || batch <= 0 || batch > 65535 || heads <= 0 || heads > DS_ATTN_MAX_HEADS) return DS_ERR_ARG;
+  if ((long)batch * ((heads + 127) / 128) > 65535) return DS_ERR_ARG;  // grid z of the weighted-sum kernel
   if (d < 64 || d > DS_ATTN_MAX_DIM || d % 64 != 0 || T <= 0 || kv_batch_stride < 0) return DS_ERR_ARG;
   if (k < 0 || k > DS_MAX_K || (k > 0 && !idx) || W < 0 || W > DS_ATTN_MAX_WINDOW || (W > 0 && !win))
     return DS_ERR_ARG;

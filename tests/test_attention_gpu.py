@@ -140,13 +140,14 @@ def test_decode_workload_full_size(cuda_device):
 
 
 def test_many_rows_run_in_pieces(cuda_device):
-    # 64 rows x 34 chunks of partial results exceed the scratch cap, so the
-    # call runs in two pieces; a sample of rows is checked
-    a = inputs.attention(seed=10, batch=64, heads=128, d=512, T=8192, k=2048, W=128, shared_cache=True,
+    # 1024 rows x 34 chunks of weight and row tiles (about 2.8 MiB a row)
+    # exceed the 512 MiB scratch cap, so the call runs in several pieces of
+    # about 180 rows; rows from several pieces are checked
+    a = inputs.attention(seed=10, batch=1024, heads=128, d=512, T=8192, k=2048, W=128, shared_cache=True,
                          vl_lo=4096, vl_hi=8192)
     scale = 1.0 / math.sqrt(512)
     out, lse = _run(a, cuda_device, scale)
-    rows = [0, 1, 30, 56, 57, 63]
+    rows = [0, 1, 181, 182, 500, 906, 907, 1023]
     sub = dict(a)
     sub["q"], sub["idx"], sub["win"], sub["win_len"] = a["q"][rows], a["idx"][rows], a["win"][rows], a["win_len"][rows]
     _check(sub, out[rows], lse[rows], scale)
