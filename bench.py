@@ -90,6 +90,80 @@ def attention_bytes_flops(idx, T, win_len, heads, d, k):
     return bytes_, flops
 
 
+def measure_attention(ds, inputs, dev, stream, rank, hbm_gbs, tflops, calls, warmup=3):
+    """Sparse attention over the selected rows (the step that consumes the
+    selection): 8 tokens x 128 heads x d = 512 against a 32768-row cache per
+    batch row, k = 1024 slots plus a window of 128.  L2 is flushed (a 256 MiB
+    write) before every timed call, so the gathered rows come from HBM as they
+    do after the selection step."""
+    import torch
+    A = ATTENTION
+    aa = inputs.attention(seed=inputs.SEED_ATTENTION + rank, batch=A["batch"], heads=A["heads"], d=A["d"],
+                          T=A["T"], k=A["k"], W=A["W"])
+    a_q = torch.from_numpy(aa["q"].view(np.int16)).view(torch.bfloat16).to(dev)
+    a_kv = torch.from_numpy(aa["kv"].view(np.int16)).view(torch.bfloat16).to(dev)
+    a_win = torch.from_numpy(aa["win"].view(np.int16)).view(torch.bfloat16).to(dev)
+    a_idx = torch.from_numpy(aa["idx"]).to(dev)
+    a_wl = torch.from_numpy(aa["win_len"]).to(dev)
+    a_sink = torch.from_numpy(aa["sink"]).to(dev)
+    a_out = torch.empty((A["batch"], A["heads"], A["d"]), dtype=torch.bfloat16, device=dev)
+    a_lse = torch.empty((A["batch"], A["heads"]), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def attn_call():
+        ds.ds_sparse_attention(a_q, a_kv, a_idx, win=a_win, win_len=a_wl, sink=a_sink, out=a_out, lse=a_lse)
+
+    for _ in range(warmup):
+        attn_call()
+    torch.cuda.synchronize()
+    barrier()
+    a_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(calls)]
+    for i in range(calls):
+        flush.fill_(float(i))
+        a_ev[i][0].record(stream)
+        attn_call()
+        a_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    attn_us = sum(e0.elapsed_time(e1) for e0, e1 in a_ev) / calls * 1e3
+    (attn_us,) = max_over_ranks([attn_us], dev)
+    del flush
+    status = ds.ds_get_device_status()
+    if status != ds.DS_OK:
+        raise RuntimeError(f"device status after attention: {ds.strerror(status)}")
+    abytes, aflops = attention_bytes_flops(aa["idx"], A["T"], aa["win_len"], A["heads"], A["d"], A["k"])
+    a_t_hbm = abytes / (hbm_gbs * 1e9) * 1e6
+    a_t_tc = aflops / (tflops * 1e12) * 1e6
+    return {
+        "workload": "8 tokens x 128 heads x d=512 bf16 queries; per-row bf16 cache of 32768 x 512; k=1024 "
+                    "selected rows + window of 128 + per-head sink; out bf16 + lse f32; L2 flushed per call",
+        "us_per_call": round(attn_us, 2),
+        "roofline_us": round(max(a_t_hbm, a_t_tc), 3),
+        "bound": "hbm" if a_t_hbm >= a_t_tc else "tensor",
+        "frac_of_roofline": round(max(a_t_hbm, a_t_tc) / attn_us, 3),
+        "achieved_gbs": round(abytes / (attn_us * 1e-6) / 1e9, 1),
+        "achieved_tflops": round(aflops / (attn_us * 1e-6) / 1e12, 1),
+        "algorithmic_bytes": int(abytes), "flops": int(aflops),
+        "peaks": {"hbm_gbs": hbm_gbs, "bf16_tflops": tflops, "kind": "burst"},
+    }
+
+
+def run_attention_only(args):
+    """`--only attention`: the sparse-attention measurement alone (the command
+    the attention profiles are taken with)."""
+    import torch
+    import sparse_attention_top_ds_b200 as ds
+    from sparse_attention_top_ds_b200 import inputs
+    rank, ws = dist_setup("nccl")
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    hbm_gbs, tflops, _, _ = load_peaks()
+    a = measure_attention(ds, inputs, dev, torch.cuda.current_stream(), rank, hbm_gbs, tflops, args.steps,
+                          warmup=args.warmup)
+    if rank == 0:
+        print(json.dumps({"sparse_attention": a, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup}),
+              flush=True)
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -408,59 +482,7 @@ def run_ours(args):
     if status != ds.DS_OK:
         raise RuntimeError(f"device status after prefill: {ds.strerror(status)}")
 
-    # ---- sparse attention over the selected rows (the step that consumes the
-    # selection), beside the headline: 8 tokens x 128 heads x d = 512 against
-    # a 32768-row cache per batch row, k = 1024 slots plus a window of 128.
-    # L2 is flushed (a 256 MiB write) before every timed call, so the gathered
-    # rows come from HBM as they do after the selection step.
-    A = ATTENTION
-    aa = inputs.attention(seed=inputs.SEED_ATTENTION + rank, batch=A["batch"], heads=A["heads"], d=A["d"],
-                          T=A["T"], k=A["k"], W=A["W"])
-    a_q = torch.from_numpy(aa["q"].view(np.int16)).view(torch.bfloat16).to(dev)
-    a_kv = torch.from_numpy(aa["kv"].view(np.int16)).view(torch.bfloat16).to(dev)
-    a_win = torch.from_numpy(aa["win"].view(np.int16)).view(torch.bfloat16).to(dev)
-    a_idx = torch.from_numpy(aa["idx"]).to(dev)
-    a_wl = torch.from_numpy(aa["win_len"]).to(dev)
-    a_sink = torch.from_numpy(aa["sink"]).to(dev)
-    a_out = torch.empty((A["batch"], A["heads"], A["d"]), dtype=torch.bfloat16, device=dev)
-    a_lse = torch.empty((A["batch"], A["heads"]), dtype=torch.float32, device=dev)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-
-    def attn_call():
-        ds.ds_sparse_attention(a_q, a_kv, a_idx, win=a_win, win_len=a_wl, sink=a_sink, out=a_out, lse=a_lse)
-
-    for _ in range(3):
-        attn_call()
-    torch.cuda.synchronize()
-    barrier()
-    a_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(ATTN_CALLS)]
-    for i in range(ATTN_CALLS):
-        flush.fill_(float(i))
-        a_ev[i][0].record(stream)
-        attn_call()
-        a_ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    attn_us = sum(e0.elapsed_time(e1) for e0, e1 in a_ev) / ATTN_CALLS * 1e3
-    (attn_us,) = max_over_ranks([attn_us], dev)
-    del flush
-    status = ds.ds_get_device_status()
-    if status != ds.DS_OK:
-        raise RuntimeError(f"device status after attention: {ds.strerror(status)}")
-    abytes, aflops = attention_bytes_flops(aa["idx"], A["T"], aa["win_len"], A["heads"], A["d"], A["k"])
-    a_t_hbm = abytes / (hbm_gbs * 1e9) * 1e6
-    a_t_tc = aflops / (tflops * 1e12) * 1e6
-    attention = {
-        "workload": "8 tokens x 128 heads x d=512 bf16 queries; per-row bf16 cache of 32768 x 512; k=1024 "
-                    "selected rows + window of 128 + per-head sink; out bf16 + lse f32; L2 flushed per call",
-        "us_per_call": round(attn_us, 2),
-        "roofline_us": round(max(a_t_hbm, a_t_tc), 3),
-        "bound": "hbm" if a_t_hbm >= a_t_tc else "tensor",
-        "frac_of_roofline": round(max(a_t_hbm, a_t_tc) / attn_us, 3),
-        "achieved_gbs": round(abytes / (attn_us * 1e-6) / 1e9, 1),
-        "achieved_tflops": round(aflops / (attn_us * 1e-6) / 1e12, 1),
-        "algorithmic_bytes": int(abytes), "flops": int(aflops),
-        "peaks": {"hbm_gbs": hbm_gbs, "bf16_tflops": tflops, "kind": "burst"},
-    }
+    attention = measure_attention(ds, inputs, dev, stream, rank, hbm_gbs, tflops, ATTN_CALLS)
 
     traffic = None
     prof = os.path.join(ROOT, "profiles", "topk_traffic.json")
@@ -523,11 +545,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["all", "attention"], default="all",
+                    help="attention: time the sparse attention alone (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.only == "attention":
+        run_attention_only(args)
     else:
         run_ours(args)
     import torch.distributed as dist

@@ -190,13 +190,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     if (ok) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, kAttnRows);
+      // the start address is the descriptor's low field (in 16-byte units), so
+      // moving through the tiles is an add on the first descriptor
+      const uint64_t a0 = sw128_kmajor_desc(q_s), b0 = sw128_kmajor_desc(kv_s);
       for (int db = 0; db < DB; ++db) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t a = sw128_kmajor_desc(q_s + (uint32_t)db * 16384u + (uint32_t)kk * 32u);
-          const uint64_t bd = sw128_kmajor_desc(kv_s + (uint32_t)db * kRowTile + (uint32_t)kk * 32u);
-          mma_bf16_ss(tmem, a, bd, idesc, (db | kk) != 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ss(tmem, a0 + (uint64_t)((db * 16384 + kk * 32) >> 4), b0 + (uint64_t)((db * kRowTile + kk * 32) >> 4),
+                      idesc, (db | kk) != 0 ? 1u : 0u);
       }
     }
     mma_commit(bar_s);  // arrives even when nothing was issued, so that no one waits for ever
@@ -433,14 +434,12 @@ __global__ void __launch_bounds__(kPvWarps * 32, 1) sparse_attn_pv_kernel(const 
       fence_proxy_async_smem();
       tc_fence_after();
       const uint32_t st = sbase + (uint32_t)s * L_::kStage;
+      const uint64_t a0 = sw128_kmajor_desc(st), b0 = sw128_mnmajor_desc(st + (uint32_t)K * kAttnTile, 8192u, 1024u);
       for (int t = 0; t < n; ++t) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t a = sw128_kmajor_desc(st + (uint32_t)t * kAttnTile + (uint32_t)kk * 32u);
-          const uint64_t bd = sw128_mnmajor_desc(st + (uint32_t)K * kAttnTile + (uint32_t)t * kRowTile +
-                                                     (uint32_t)kk * 2048u, 8192u, 1024u);
-          mma_bf16_ss(tmem, a, bd, idesc, (j | t | kk) != 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ss(tmem, a0 + (uint64_t)((t * kAttnTile + kk * 32) >> 4), b0 + (uint64_t)((t * kRowTile + kk * 2048) >> 4),
+                      idesc, (j | t | kk) != 0 ? 1u : 0u);
       }
       mma_commit(empty0 + 8u * s);
     }
