@@ -18,6 +18,10 @@ selection step computes, in float64:
                     rows plus a sliding window (NKI pull request, steps table
                     row 4 "Concatenate and attend"), with an optional per-head
                     attention sink.
+* ``qproj``      -- the indexer query projection: q = x . Wq^T into 128
+                    channels per head, rounded to bfloat16, and the per-head
+                    weights w = x . Ww^T (NKI pull request, steps table row 2
+                    and the launch list's query-projection GEMV).
 * ``indexer``    -- the lightning-indexer score
                     ``score[t,s] = sum_h w[t,h] * max(0, q[t,h,:] . k[s,:])``
                     (NKI pull request "Add DeepSeek-V4 CSA attention kernels",
@@ -33,8 +37,9 @@ from .encoding import decode_bf16, decode_f32, NEG_INF_BF16, NEG_INF_F32
 from .topk import topk_rows, topk_row
 from .indexer import indexer_scores, indexer_topk
 from .attention import sparse_attention
+from .qproj import qproj, round_bf16
 
 __all__ = [
     "decode_bf16", "decode_f32", "NEG_INF_BF16", "NEG_INF_F32",
-    "topk_rows", "topk_row", "indexer_scores", "indexer_topk", "sparse_attention",
+    "topk_rows", "topk_row", "indexer_scores", "indexer_topk", "sparse_attention", "qproj", "round_bf16",
 ]
