@@ -9,9 +9,11 @@ seeded input:
     and indices, unsorted;
   * the decode indexer + top-k (8 query rows x 64 heads x 128 bf16 against one
     bf16 key cache of 32768 positions, valid_len ~ U{4096..32768}, k = 1024).
-Reported beside it: the prefill indexer + top-k, and the sparse attention that
+Reported beside it: the prefill indexer + top-k; the sparse attention that
 consumes the selection (8 tokens x 128 heads x 512 over k = 1024 selected rows
-plus a window of 128, L2 flushed before each call).
+plus a window of 128, rotating slot sets); and the indexer query
+projection that feeds the scorer (8 tokens, width 1536 -> 64 x 128 queries and
+64 weights), alone and chained in front of the decode indexer + top-k.
 The headline value is the top-k effective HBM bandwidth (algorithmic bytes /
 device time, GB/s); the decode indexer + top-k time is reported in
 microseconds per decode step beside it.  Inputs rotate through enough copies
@@ -50,6 +52,7 @@ DECODE = dict(batch=8, heads=64, d=128, S=32768, k=1024)
 PREFILL = dict(k=2048)
 ATTENTION = dict(batch=8, heads=128, d=512, T=32768, k=1024, W=128)
 ATTN_CALLS = 40
+QPROJ = dict(T=8, d_in=1536, heads=64)
 
 
 def load_peaks():
@@ -90,52 +93,75 @@ def attention_bytes_flops(idx, T, win_len, heads, d, k):
     return bytes_, flops
 
 
+def graph_time_us(fn_of_i, count, reps=3):
+    """Device time per call of fn_of_i(0..count-1), captured as one CUDA graph
+    (host launch cost off the device timeline) and replayed `reps` times after
+    one warm replay; CUDA events on the current stream."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for i in range(count):          # warm-up, and the first-use set-up of each input set
+        fn_of_i(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(count):
+            fn_of_i(i)
+    g.replay()
+    torch.cuda.synchronize()
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) * 1e3 / (count * reps)
+
+
 def measure_attention(ds, inputs, dev, stream, rank, hbm_gbs, tflops, calls, warmup=3):
     """Sparse attention over the selected rows (the step that consumes the
     selection): 8 tokens x 128 heads x d = 512 against a 32768-row cache per
-    batch row, k = 1024 slots plus a window of 128.  L2 is flushed (a 256 MiB
-    write) before every timed call, so the gathered rows come from HBM as they
-    do after the selection step."""
+    batch row, k = 1024 slots plus a window of 128.  Calls rotate through 24
+    slot sets, each with its own copy of the queries and the window, so that
+    between two uses of a set the other sets have touched more than 2x L2 of
+    rows: every call gathers its rows from HBM, as after the selection step."""
     import torch
     A = ATTENTION
+    R = 24
     aa = inputs.attention(seed=inputs.SEED_ATTENTION + rank, batch=A["batch"], heads=A["heads"], d=A["d"],
                           T=A["T"], k=A["k"], W=A["W"])
-    a_q = torch.from_numpy(aa["q"].view(np.int16)).view(torch.bfloat16).to(dev)
-    a_kv = torch.from_numpy(aa["kv"].view(np.int16)).view(torch.bfloat16).to(dev)
-    a_win = torch.from_numpy(aa["win"].view(np.int16)).view(torch.bfloat16).to(dev)
-    a_idx = torch.from_numpy(aa["idx"]).to(dev)
+    to = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    a_kv = to(aa["kv"])
+    q0, w0 = to(aa["q"]), to(aa["win"])
+    a_q = [q0.clone() for _ in range(R)]
+    a_win = [w0.clone() for _ in range(R)]
+    idx_sets = [aa["idx"]] + [inputs.attention_slots(inputs.SEED_ATTENTION + 1000 * (rank + 1) + r, batch=A["batch"],
+                                                     T=A["T"], k=A["k"]) for r in range(1, R)]
+    a_idx = [torch.from_numpy(i).to(dev) for i in idx_sets]
     a_wl = torch.from_numpy(aa["win_len"]).to(dev)
     a_sink = torch.from_numpy(aa["sink"]).to(dev)
     a_out = torch.empty((A["batch"], A["heads"], A["d"]), dtype=torch.bfloat16, device=dev)
     a_lse = torch.empty((A["batch"], A["heads"]), dtype=torch.float32, device=dev)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
-    def attn_call():
-        ds.ds_sparse_attention(a_q, a_kv, a_idx, win=a_win, win_len=a_wl, sink=a_sink, out=a_out, lse=a_lse)
+    def call(i):
+        r = i % R
+        ds.ds_sparse_attention(a_q[r], a_kv, a_idx[r], win=a_win[r], win_len=a_wl, sink=a_sink, out=a_out, lse=a_lse)
 
-    for _ in range(warmup):
-        attn_call()
-    torch.cuda.synchronize()
-    barrier()
-    a_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(calls)]
-    for i in range(calls):
-        flush.fill_(float(i))
-        a_ev[i][0].record(stream)
-        attn_call()
-        a_ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    attn_us = sum(e0.elapsed_time(e1) for e0, e1 in a_ev) / calls * 1e3
+    attn_us = graph_time_us(call, R, reps=max(1, calls // R))
     (attn_us,) = max_over_ranks([attn_us], dev)
-    del flush
     status = ds.ds_get_device_status()
     if status != ds.DS_OK:
         raise RuntimeError(f"device status after attention: {ds.strerror(status)}")
-    abytes, aflops = attention_bytes_flops(aa["idx"], A["T"], aa["win_len"], A["heads"], A["d"], A["k"])
+    ab = [attention_bytes_flops(i, A["T"], aa["win_len"], A["heads"], A["d"], A["k"]) for i in idx_sets]
+    abytes = sum(x[0] for x in ab) / R
+    aflops = sum(x[1] for x in ab) / R
     a_t_hbm = abytes / (hbm_gbs * 1e9) * 1e6
     a_t_tc = aflops / (tflops * 1e12) * 1e6
     return {
         "workload": "8 tokens x 128 heads x d=512 bf16 queries; per-row bf16 cache of 32768 x 512; k=1024 "
-                    "selected rows + window of 128 + per-head sink; out bf16 + lse f32; L2 flushed per call",
+                    "selected rows + window of 128 + per-head sink; out bf16 + lse f32; 24 rotating slot sets "
+                    "(> 2x L2 of rows between reuses)",
         "us_per_call": round(attn_us, 2),
         "roofline_us": round(max(a_t_hbm, a_t_tc), 3),
         "bound": "hbm" if a_t_hbm >= a_t_tc else "tensor",
@@ -147,9 +173,58 @@ def measure_attention(ds, inputs, dev, stream, rank, hbm_gbs, tflops, calls, war
     }
 
 
+def measure_qproj(ds, inputs, dev, stream, rank, hbm_gbs, calls, warmup=3):
+    """The indexer query projection of a decode step (8 tokens, width 1536,
+    64 heads x 128 + 64 per-head weights), alone and chained in front of the
+    decode indexer + top-k.  Calls rotate through 11 copies of the 25.5 MB of
+    weights (and 33 copies of the 8 MB key cache for the chained step), more
+    than 2x L2 between reuses, so the weights come from HBM."""
+    import torch
+    Q = QPROJ
+    x, wq, ww = inputs.qproj(seed=inputs.SEED_QPROJ + rank, T=Q["T"], d_in=Q["d_in"], heads=Q["heads"])
+    to = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    xd = to(x)
+    Rw = max(3, -(-2 * L2_BYTES // (wq.nbytes + ww.nbytes)) + 1)
+    wq0, ww0 = to(wq), to(ww)
+    wqs = [wq0] + [wq0.clone() for _ in range(Rw - 1)]
+    wws = [ww0] + [ww0.clone() for _ in range(Rw - 1)]
+    q_out = torch.empty((Q["T"], Q["heads"], 128), dtype=torch.bfloat16, device=dev)
+    w_out = torch.empty((Q["T"], Q["heads"]), dtype=torch.float32, device=dev)
+    _, kc, _, vl = inputs.decode(seed=inputs.SEED_DECODE + rank)
+    Rk = max(3, -(-2 * L2_BYTES // kc.nbytes) + 1)
+    kc0 = to(kc)
+    kcs = [kc0] + [kc0.clone() for _ in range(Rk - 1)]
+    vld = torch.from_numpy(vl).to(dev)
+    idx = torch.empty((Q["T"], DECODE["k"]), dtype=torch.int32, device=dev)
+
+    def proj(i):
+        ds.ds_indexer_qproj(xd, wqs[i % Rw], wws[i % Rw], q_out=q_out, w_out=w_out)
+
+    def step(i):
+        proj(i)
+        ds.ds_indexer_topk(q_out, kcs[i % Rk], w_out, DECODE["k"], valid_len=vld, out_idx=idx)
+
+    proj_us = graph_time_us(proj, Rw, reps=max(1, calls // Rw))
+    step_us = graph_time_us(step, Rk, reps=max(1, calls // Rk))
+    proj_us, step_us = max_over_ranks([proj_us, step_us], dev)
+    status = ds.ds_get_device_status()
+    if status != ds.DS_OK:
+        raise RuntimeError(f"device status after the projection: {ds.strerror(status)}")
+    nbytes = wq.nbytes + ww.nbytes + x.nbytes + q_out.numel() * 2 + w_out.numel() * 4
+    roof_us = nbytes / (hbm_gbs * 1e9) * 1e6
+    return {
+        "workload": f"8 tokens x width 1536 bf16 -> 64 heads x 128 bf16 queries + 64 f32 weights "
+                    f"(Wq 8192 x 1536, Ww 64 x 1536 bf16); {Rw} rotating weight copies (> 2x L2 between reuses)",
+        "us_per_call": round(proj_us, 2), "roofline_us": round(roof_us, 3), "bound": "hbm",
+        "frac_of_roofline": round(roof_us / proj_us, 3),
+        "achieved_gbs": round(nbytes / (proj_us * 1e-6) / 1e9, 1), "algorithmic_bytes": int(nbytes),
+        "decode_step_with_projection_us": round(step_us, 2),
+    }
+
+
 def run_attention_only(args):
-    """`--only attention`: the sparse-attention measurement alone (the command
-    the attention profiles are taken with)."""
+    """`--only attention` / `--only qproj`: one beside-the-headline measurement
+    alone (the commands the profiles of those kernels are taken with)."""
     import torch
     import sparse_attention_top_ds_b200 as ds
     from sparse_attention_top_ds_b200 import inputs
@@ -157,11 +232,14 @@ def run_attention_only(args):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
     hbm_gbs, tflops, _, _ = load_peaks()
-    a = measure_attention(ds, inputs, dev, torch.cuda.current_stream(), rank, hbm_gbs, tflops, args.steps,
-                          warmup=args.warmup)
+    stream = torch.cuda.current_stream()
+    if args.only == "qproj":
+        key, a = "qproj", measure_qproj(ds, inputs, dev, stream, rank, hbm_gbs, args.steps, warmup=args.warmup)
+    else:
+        key, a = "sparse_attention", measure_attention(ds, inputs, dev, stream, rank, hbm_gbs, tflops, args.steps,
+                                                       warmup=args.warmup)
     if rank == 0:
-        print(json.dumps({"sparse_attention": a, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup}),
-              flush=True)
+        print(json.dumps({key: a, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup}), flush=True)
 
 
 # ------------------------------------------------------------------ clocks
@@ -483,6 +561,7 @@ def run_ours(args):
         raise RuntimeError(f"device status after prefill: {ds.strerror(status)}")
 
     attention = measure_attention(ds, inputs, dev, stream, rank, hbm_gbs, tflops, ATTN_CALLS)
+    qproj = measure_qproj(ds, inputs, dev, stream, rank, hbm_gbs, ATTN_CALLS)
 
     traffic = None
     prof = os.path.join(ROOT, "profiles", "topk_traffic.json")
@@ -527,6 +606,7 @@ def run_ours(args):
                         "scorer_frac_of_bf16_peak": round(pre_flops / (pre_score_ms * 1e-3) / 1e12 / tflops_sus, 3),
                         "bf16_peak_tflops": tflops_sus, "peak_kind": "sustained"},
             "sparse_attention": attention,
+            "qproj": qproj,
             "roofline": {"bound": "hbm", "achieved": round(per_launch_gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
                          "frac": round(per_launch_gbs / hbm_gbs, 4), "traffic": traffic,
                          "kernel": TOPK_KERNEL, "peak_source": peak_src},
@@ -545,14 +625,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "attention"], default="all",
-                    help="attention: time the sparse attention alone (profiling)")
+    ap.add_argument("--only", choices=["all", "attention", "qproj"], default="all",
+                    help="time the sparse attention or the query projection alone (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
-    elif args.only == "attention":
+    elif args.only in ("attention", "qproj"):
         run_attention_only(args)
     else:
         run_ours(args)

@@ -2,7 +2,7 @@
  * ds_topk.h -- C ABI of libdstopk.so, the selection step of DeepSeek-style
  * sparse attention on B200 (sm_100a).
  *
- * Three operations, as described on the pages this library follows:
+ * Four operations, as described on the pages this library follows:
  *
  *  - Row-wise top-k of given scores (DeepSelect hub page, use-case paragraphs:
  *    pick the top-k positions of every score row; bfloat16 rows for the
@@ -15,6 +15,9 @@
  *        score[t,s] = sum_h w[t,h] * max(0, q[t,h,:] . k[s,:])
  *    over a 128-channel bfloat16 key cache shared by all rows, then the k
  *    highest-scoring positions of each row.
+ *
+ *  - The indexer query projection that produces the scorer's queries and
+ *    per-head weights (the same pull request, steps table row 2).
  *
  *  - The attention that consumes the selection (the same pull request, steps
  *    table row 4): multi-query softmax attention of every query head over
@@ -169,6 +172,35 @@ int ds_indexer_topk_noalloc(const void* q, const void* kcache, const float* w,
                             int batch, int heads, int d, int S,
                             const int32_t* valid_len, int k,
                             int32_t* out_idx, float* out_score, void* stream);
+
+/*
+ * ds_indexer_qproj -- the indexer query projection: the per-head queries and
+ * weights that ds_indexer_score / ds_indexer_topk take, from one input vector
+ * per token.
+ *   (NKI pull request "Add DeepSeek-V4 CSA attention kernels", "How the
+ *    algorithm works", steps table row 2: the indexer query is projected into
+ *    128 channels; launch list: the query projection runs as a GEMV ahead of
+ *    the scoring launch.)
+ *
+ *     q[t, h, c] = sum_i x[t, i] * wq[h * d + c, i]    rounded to bfloat16
+ *     w[t, h]    = sum_i x[t, i] * ww[h, i]             float32
+ *
+ * x       device bfloat16 [T, d_in]; 16-byte aligned.
+ * wq      device bfloat16 [heads * d, d_in] (row-major, one row per output
+ *         channel); 16-byte aligned.
+ * ww      device bfloat16 [heads, d_in] or NULL; 16-byte aligned.
+ * T       1 .. 524280 tokens (decode batches are the intended use: every group
+ *         of 8 tokens streams the weights once).
+ * d_in    a multiple of 8, 8 <= d_in <= 8192.
+ * heads   1 .. DS_INDEXER_MAX_HEADS;  d == DS_INDEXER_DIM.
+ * q_out   device bfloat16 [T, heads, d] (the layout ds_indexer_topk reads).
+ * w_out   device float32 [T, heads]; must be NULL exactly when ww is NULL.
+ * The products of the exact bfloat16 inputs are accumulated in float32 on the
+ * CUDA cores (packed two-lane FMAs); q is rounded to the nearest bfloat16.
+ * Returns DS_OK, DS_ERR_ARG, DS_ERR_UNSUPPORTED or DS_ERR_CUDA.
+ */
+int ds_indexer_qproj(const void* x, const void* wq, const void* ww, int T, int d_in, int heads, int d,
+                     void* q_out, float* w_out, void* stream);
 
 /*
  * ds_sparse_attention -- multi-query decode attention over the selected

@@ -63,6 +63,8 @@ def load():
     lib.ds_sparse_attention.argtypes = [vp, vp, ctypes.c_int64, i32, i32p, i32, vp, i32, i32p, vp,
                                         i32, i32, i32, ctypes.c_float, vp, vp, vp]
     lib.ds_sparse_attention.restype = i32
+    lib.ds_indexer_qproj.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp]
+    lib.ds_indexer_qproj.restype = i32
     lib.ds_get_device_status.argtypes = [vp]
     lib.ds_get_device_status.restype = i32
     lib.ds_strerror.argtypes = [i32]
@@ -107,6 +109,10 @@ def ds_sparse_attention_raw(q, kv, kv_batch_stride, T, idx, k, win, W, win_len, 
                             out, lse, stream):
     return load().ds_sparse_attention(q, kv, int(kv_batch_stride), T, idx, k, win, W, win_len, sink,
                                       batch, heads, d, float(scale), out, lse, stream)
+
+
+def ds_indexer_qproj_raw(x, wq, ww, T, d_in, heads, d, q_out, w_out, stream):
+    return load().ds_indexer_qproj(x, wq, ww, T, d_in, heads, d, q_out, w_out, stream)
 
 
 def ds_get_device_status(stream=None):
@@ -287,3 +293,35 @@ def ds_sparse_attention(q, kv, idx, scale=None, win=None, win_len=None, sink=Non
                                      _stream_ptr(stream))
     _check(rc, "ds_sparse_attention")
     return (out, lse) if return_lse else out
+
+
+def ds_indexer_qproj(x, wq, ww=None, heads=None, q_out=None, w_out=None, stream=None):
+    """Indexer queries and per-head weights from one input row per token.
+
+    x bf16 [T, d_in];  wq bf16 [heads * 128, d_in];  ww bf16 [heads, d_in] or None.
+    Returns (q bf16 [T, heads, 128], w float32 [T, heads] or None).
+    """
+    import torch
+    _require(x, torch.bfloat16, "x")
+    dev = x.device
+    _require(wq, torch.bfloat16, "wq", dev)
+    if x.dim() != 2 or wq.dim() != 2 or wq.shape[1] != x.shape[1] or wq.shape[0] % DS_INDEXER_DIM:
+        raise ValueError("x [T, d_in], wq [heads * 128, d_in]")
+    T, d_in = x.shape
+    H = wq.shape[0] // DS_INDEXER_DIM if heads is None else int(heads)
+    if ww is not None:
+        _require(ww, torch.bfloat16, "ww", dev)
+        if tuple(ww.shape) != (H, d_in):
+            raise ValueError("ww must be [heads, d_in]")
+    if q_out is None:
+        q_out = torch.empty((T, H, DS_INDEXER_DIM), dtype=torch.bfloat16, device=dev)
+    _require(q_out, torch.bfloat16, "q_out", dev)
+    if ww is not None and w_out is None:
+        w_out = torch.empty((T, H), dtype=torch.float32, device=dev)
+    if w_out is not None:
+        _require(w_out, torch.float32, "w_out", dev)
+    with torch.cuda.device(dev):
+        rc = ds_indexer_qproj_raw(_ptr(x), _ptr(wq), _ptr(ww), T, d_in, H, DS_INDEXER_DIM, _ptr(q_out),
+                                  _ptr(w_out) if ww is not None else None, _stream_ptr(stream))
+    _check(rc, "ds_indexer_qproj")
+    return q_out, (w_out if ww is not None else None)

@@ -19,6 +19,7 @@
 #include "decode_kernel.cuh"
 #include "rowcluster_kernel.cuh"
 #include "attention_kernel.cuh"
+#include "qproj_kernel.cuh"
 
 namespace dstopk {
 
@@ -318,6 +319,11 @@ static cudaError_t indexer_setup() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(sparse_attn_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnSmem::bytes(kAttnMaxD));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(indexer_qproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kQpTok * kQpMaxIn * 2 + 8 * 32 * 33 * 4);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(indexer_qproj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, QtSmem::kBytes);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(sparse_attn_pv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   if (e == cudaSuccess)
@@ -721,6 +727,67 @@ static int attention_enqueue(const uint16_t* q, const uint16_t* kv, long long kv
   return DS_OK;
 }
 
+// ---- indexer query projection on the tensor cores (input width a multiple of 64)
+
+// A [rows][d_in] bf16 matrix viewed as (64 channels, rows, d_in/64 blocks), in
+// boxes of (64, box_rows, bpb): rows block by block, 128-byte swizzle.
+static bool encode_rowblocks(const void* base, long long rows, int d_in, int box_rows, int bpb, CUtensorMap* m) {
+  cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(d_in / 64)};
+  cuuint64_t str[2] = {(cuuint64_t)d_in * 2, 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)bpb};
+  cuuint32_t one[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, str, box, one,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int qproj_tc_enqueue(const void* x, const void* wq, const void* ww, int T, int d_in, int heads, int d,
+                            void* q_out, float* w_out, cudaStream_t st, DeviceState* s) {
+  const int nq = heads * d;
+  const int nqb = nq / 128;
+  const int nrb = nqb + (ww ? 1 : 0);
+  const int nblk = d_in / 64;
+  const int ntg = (T + kQtTok - 1) / kQtTok;
+  // split the input width over a cluster pair while one CTA per row block
+  // would leave more than half of the SMs idle
+  const int G = (nblk % 2 == 0 && 2 * nrb * ntg <= s->num_sms) ? 2 : 1;
+  const int per = nblk / G;
+  const int bpb = per % 4 == 0 ? 4 : 1;
+  CUtensorMap twq, tww, tx;
+  if (!encode_rowblocks(wq, nq, d_in, 128, bpb, &twq)) return DS_ERR_ARG;
+  if (!encode_rowblocks(ww ? ww : wq, ww ? heads : nq, d_in, 128, bpb, &tww)) return DS_ERR_ARG;
+  if (!encode_rowblocks(x, T, d_in, kQtTok, bpb, &tx)) return DS_ERR_ARG;
+  QtParams p;
+  p.q = static_cast<uint16_t*>(q_out);
+  p.w = w_out;
+  p.status = s->status;
+  p.T = T;
+  p.nq = nq;
+  p.heads = heads;
+  p.nblk = nblk;
+  p.bpb = bpb;
+  p.nqb = nqb;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)nrb, (unsigned)G, (unsigned)ntg);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)QtSmem::kBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl_on()) set_pdl(attr[na++]);
+  if (G == 2) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = 2;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, indexer_qproj_tc_kernel, twq, tww, tx, p) == cudaSuccess ? DS_OK : DS_ERR_CUDA;
+}
+
 }  // namespace dstopk
 
 using namespace dstopk;
@@ -896,4 +963,42 @@ extern "C" int ds_sparse_attention(const void* q, const void* kv, int64_t kv_bat
   return attention_enqueue(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(kv), (long long)kv_batch_stride,
                            T, idx, k, static_cast<const uint16_t*>(win), W, win_len, sink, batch, heads, d, scale,
                            static_cast<uint16_t*>(out), lse, static_cast<cudaStream_t>(stream), s);
+}
+
+extern "C" int ds_indexer_qproj(const void* x, const void* wq, const void* ww, int T, int d_in, int heads, int d,
+                                void* q_out, float* w_out, void* stream) {
+  auto misaligned = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; };
+  if (!x || !wq || !q_out || (ww == nullptr) != (w_out == nullptr)) return DS_ERR_ARG;
+  if (T <= 0 || T > 65535 * kQpTok || heads <= 0 || heads > DS_INDEXER_MAX_HEADS || d != DS_INDEXER_DIM) return DS_ERR_ARG;
+  if (d_in < 8 || d_in > kQpMaxIn || d_in % 8 != 0) return DS_ERR_ARG;
+  if (misaligned(x, 16) || misaligned(wq, 16) || (ww && misaligned(ww, 16)) || misaligned(q_out, 2) ||
+      (w_out && misaligned(w_out, 4)))
+    return DS_ERR_ARG;
+  DeviceState* s = nullptr;
+  const int rc = device_state(&s);
+  if (rc != DS_OK) return rc;
+  if (d_in % 64 == 0) return qproj_tc_enqueue(x, wq, ww, T, d_in, heads, d, q_out, w_out, static_cast<cudaStream_t>(stream), s);
+  QpParams p;
+  p.x = static_cast<const uint16_t*>(x);
+  p.wq = static_cast<const uint16_t*>(wq);
+  p.ww = static_cast<const uint16_t*>(ww);
+  p.q = static_cast<uint16_t*>(q_out);
+  p.w = w_out;
+  p.T = T;
+  p.d_in = d_in;
+  p.heads = heads;
+  p.nq = heads * d;
+  p.nrows = p.nq + (ww ? heads : 0);
+  const int ntasks = (p.nrows + kQpRows - 1) / kQpRows;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)std::min((ntasks + 7) / 8, s->num_sms), (unsigned)((T + kQpTok - 1) / kQpTok), 1);
+  cfg.blockDim = dim3(kQpThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)kQpTok * d_in * 2 + 8 * 32 * 33 * 4;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  set_pdl(attr[0]);
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_on() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, indexer_qproj_kernel, p) == cudaSuccess ? DS_OK : DS_ERR_CUDA;
 }

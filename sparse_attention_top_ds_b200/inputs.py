@@ -17,6 +17,10 @@ Workloads (sizes and distributions of the selection step's headline cases):
 * ``prefill``         4096 query rows x 64 heads x 128 against 32768 keys with
                       the causal prefix valid_len[t] = floor((t + c) / 4),
                       c = 4 * (S - T/4).
+* ``qproj``           the indexer query projection of a decode step: 8 token
+                      rows of width 1536, Wq [64 x 128, 1536] ~ N(0, 1/(128 * 1536))
+                      (so q ~ N(0, 1/128), the indexer configs' query scale) and
+                      Ww [64, 1536] ~ N(0, 1/1536).
 * ``attention``       sparse-attention decode: 8 new tokens x 128 query heads x
                       head_dim 512, one compressed KV cache of 32768 rows per
                       batch row, k = 1024 selected rows drawn below a valid
@@ -35,6 +39,7 @@ SEED_INDEXER = 1003
 SEED_DECODE = 1004
 SEED_PREFILL = 1005
 SEED_ATTENTION = 1006
+SEED_QPROJ = 1007
 
 
 def rng(seed):
@@ -162,3 +167,28 @@ def attention(seed=SEED_ATTENTION, batch=8, heads=128, d=512, T=32768, k=1024, W
     wl = np.full(batch, W, dtype=np.int32) if win_len is None else np.asarray(win_len, dtype=np.int32)
     sk = g.standard_normal(heads).astype(np.float32) if sink else None
     return dict(q=q, kv=kv, win=win, idx=idx, win_len=wl, sink=sk)
+
+
+def qproj(seed=SEED_QPROJ, T=8, d_in=1536, heads=64, d=128, with_w=True):
+    """Projection inputs: (x [T, d_in], wq [heads * d, d_in], ww [heads, d_in] or None),
+    bfloat16 patterns of x ~ N(0, 1), wq ~ N(0, 1/(d * d_in)), ww ~ N(0, 1/d_in)."""
+    g = rng(seed)
+    x = f32_to_bf16_bits(g.standard_normal((T, d_in), dtype=np.float32))
+    wq = f32_to_bf16_bits(g.standard_normal((heads * d, d_in), dtype=np.float32) * np.float32(1.0 / np.sqrt(d * d_in)))
+    ww = None
+    if with_w:
+        ww = f32_to_bf16_bits(g.standard_normal((heads, d_in), dtype=np.float32) * np.float32(1.0 / np.sqrt(d_in)))
+    return x, wq, ww
+
+
+def attention_slots(seed, batch=8, T=32768, k=1024, vl_lo=4096, vl_hi=32768):
+    """Another draw of the attention workload's slots alone (int32 [batch, k]),
+    with the same rule as ``attention``: distinct rows below a valid length
+    ~ U{vl_lo..vl_hi}, -1 past it."""
+    g = rng(seed)
+    idx = np.full((batch, k), -1, dtype=np.int32)
+    for b in range(batch):
+        L = int(min(T, g.integers(min(vl_lo, T), min(vl_hi, T), endpoint=True)))
+        m = min(k, L)
+        idx[b, :m] = g.choice(L, size=m, replace=False)
+    return idx

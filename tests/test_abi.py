@@ -29,8 +29,8 @@ def declared_entry_points():
 
 def test_header_declares_the_boundary():
     names = declared_entry_points()
-    for n in ("ds_topk", "ds_indexer_score", "ds_indexer_topk", "ds_sparse_attention", "ds_get_device_status",
-              "ds_strerror", "ds_release"):
+    for n in ("ds_topk", "ds_indexer_score", "ds_indexer_topk", "ds_indexer_qproj", "ds_sparse_attention",
+              "ds_get_device_status", "ds_strerror", "ds_release"):
         assert n in names
 
 
@@ -112,6 +112,34 @@ def test_attention_argument_errors_need_no_gpu(lib):
     assert call(out=vp(0x100002)) == -1
     assert call(W=8, win=vp(0x100008)) == -1
     assert call(lse=vp(0x100002)) == -1
+
+
+def test_qproj_argument_errors_need_no_gpu(lib):
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    f = lib.ds_indexer_qproj
+    f.restype = i32
+    f.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp]
+    a = vp(0x100000)
+
+    def call(x=a, wq=a, ww=a, T=8, d_in=1536, H=64, d=128, q=a, w=a):
+        return f(x, wq, ww, T, d_in, H, d, q, w, None)
+
+    assert call(x=None) == -1
+    assert call(wq=None) == -1
+    assert call(q=None) == -1
+    assert call(ww=None) == -1            # w_out without ww
+    assert call(w=None) == -1             # ww without w_out
+    assert call(T=0) == -1
+    assert call(H=65) == -1
+    assert call(H=0) == -1
+    assert call(d=64) == -1
+    assert call(d_in=1532) == -1          # not a multiple of 8
+    assert call(d_in=8200) == -1
+    assert call(d_in=0) == -1
+    assert call(x=vp(0x100008)) == -1     # 16-byte alignment
+    assert call(wq=vp(0x100004)) == -1
+    assert call(q=vp(0x100001)) == -1
+    assert call(w=vp(0x100002)) == -1
 
 
 def test_binding_fails_loudly_without_the_library(tmp_path):
