@@ -14,7 +14,9 @@ inputs.  Readings where the pages are silent (listed in the design doc):
     then the heads are summed (the order the steps table names them in);
   * there is no extra scale factor (any scale folds into w);
   * w is per token and head, of any sign;
-  * one key cache [S, d] is shared by every query row;
+  * one key cache [S, d] is shared by every query row, or each row has its own
+    [S, d] cache (the [B, T_c, index_head_dim] indexer cache of "Launching a
+    full block");
   * positions at or beyond valid_len[t] are not scored and never selected.
 """
 
@@ -28,7 +30,8 @@ def indexer_scores(q_bits, k_bits, w, valid_len=None):
     """float64 score rows.
 
     ``q_bits`` [batch, heads, d] bfloat16 patterns (uint16);
-    ``k_bits`` [S, d] bfloat16 patterns (uint16);
+    ``k_bits`` [S, d] bfloat16 patterns (uint16), one key cache shared by every
+               row, or [batch, S, d], one cache per row;
     ``w``      [batch, heads] float32 (or float64) weights;
     ``valid_len`` None or [batch] prefix lengths.
     Returns [batch, S] float64 with NaN at positions s >= valid_len[t]
@@ -39,13 +42,15 @@ def indexer_scores(q_bits, k_bits, w, valid_len=None):
     wa = np.asarray(w)
     w64 = decode_f32(wa) if wa.dtype == np.float32 else wa.astype(np.float64)
     batch, heads, d = q.shape
-    S = kc.shape[0]
-    if kc.shape[1] != d or w64.shape != (batch, heads):
+    per_row = kc.ndim == 3
+    S = kc.shape[-2]
+    if kc.shape[-1] != d or w64.shape != (batch, heads) or (per_row and kc.shape[0] != batch):
         raise ValueError("shape mismatch")
     out = np.full((batch, S), np.nan, dtype=np.float64)
     for t in range(batch):
         L = S if valid_len is None else max(0, min(int(valid_len[t]), S))
-        dots = q[t] @ kc[:L].T                  # [heads, L]: per-head dot products
+        keys = kc[t] if per_row else kc
+        dots = q[t] @ keys[:L].T                # [heads, L]: per-head dot products
         relu = np.maximum(dots, 0.0)            # ReLU on each head's product
         out[t, :L] = (w64[t][:, None] * relu).sum(axis=0)   # weight, then sum heads
     return out

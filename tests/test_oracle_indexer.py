@@ -175,3 +175,18 @@ def test_worked_example_catches_planted_mistakes(mutant):
         if got.shape != (5,) or not np.array_equal(got, np.array(case["scores"])):
             wrong = True
     assert wrong
+
+
+def test_per_row_caches_equal_one_cache_per_call():
+    q, keys, w = _random_case(27, batch=3, S=200)
+    g = np.random.default_rng(3)
+    kc3 = np.stack([keys, keys[g.permutation(200)], keys[::-1].copy()])
+    vl = np.array([200, 57, 130])
+    got = indexer_scores(q, kc3, w, vl)
+    for t in range(3):
+        one = indexer_scores(q[t:t + 1], kc3[t], w[t:t + 1], vl[t:t + 1])
+        assert np.array_equal(np.nan_to_num(got[t], nan=-1.0), np.nan_to_num(one[0], nan=-1.0))
+    idx, _ = indexer_topk(q, kc3, w, 20, vl)
+    for t in range(3):
+        i1, _ = indexer_topk(q[t:t + 1], kc3[t], w[t:t + 1], 20, vl[t:t + 1])
+        assert idx[t].tolist() == i1[0].tolist()
