@@ -146,6 +146,27 @@ int ds_indexer_topk(const void* q, const void* kcache, const float* w,
                     int32_t* out_idx, float* out_score, void* stream);
 
 /*
+ * ds_indexer_topk_ex -- ds_indexer_topk with a key cache per row and
+ * position-sorted output.
+ *   (NKI pull request "Add DeepSeek-V4 CSA attention kernels", "Launching a
+ *    full block": the indexer key cache is [B, T_c, index_head_dim], one per
+ *    batch row; DeepSelect hub page, options paragraph: sorted_index.)
+ *
+ * kcache_batch_stride  0: kcache is one [S, d] cache shared by every row (as
+ *            in ds_indexer_topk); otherwise row t reads the S x d cache that
+ *            starts t * kcache_batch_stride rows after kcache, and the stride
+ *            must be >= S (for example S for a [batch, S, d] array).
+ * sorted_index 0 or 1: with 1 each row's selection is in ascending position
+ *            order (the selection itself is the same).
+ * The other arguments, outputs and results are those of ds_indexer_topk,
+ * including its use of the scratch buffer; this entry point always runs the
+ * scorer and the top-k as two launches.
+ */
+int ds_indexer_topk_ex(const void* q, const void* kcache, int64_t kcache_batch_stride, const float* w,
+                       int batch, int heads, int d, int S, const int32_t* valid_len, int k,
+                       int sorted_index, int32_t* out_idx, float* out_score, void* stream);
+
+/*
  * ds_indexer_topk_noalloc -- ds_indexer_topk for callers that must not
  * allocate device memory.
  *   (The pages have no counterpart: this is a deployment variant of the same

@@ -63,6 +63,8 @@ def load():
     lib.ds_sparse_attention.argtypes = [vp, vp, ctypes.c_int64, i32, i32p, i32, vp, i32, i32p, vp,
                                         i32, i32, i32, ctypes.c_float, vp, vp, vp]
     lib.ds_sparse_attention.restype = i32
+    lib.ds_indexer_topk_ex.argtypes = [vp, vp, ctypes.c_int64, vp, i32, i32, i32, i32, i32p, i32, i32, vp, vp, vp]
+    lib.ds_indexer_topk_ex.restype = i32
     lib.ds_indexer_qproj.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp]
     lib.ds_indexer_qproj.restype = i32
     lib.ds_get_device_status.argtypes = [vp]
@@ -325,3 +327,36 @@ def ds_indexer_qproj(x, wq, ww=None, heads=None, q_out=None, w_out=None, stream=
                                   _ptr(w_out) if ww is not None else None, _stream_ptr(stream))
     _check(rc, "ds_indexer_qproj")
     return q_out, (w_out if ww is not None else None)
+
+
+def ds_indexer_topk_ex(q, kcache, w, k, valid_len=None, sorted_index=False, return_score=False,
+                       out_idx=None, out_score=None, stream=None):
+    """ds_indexer_topk with kcache [S, d] (shared) or [batch, S, d] (one cache per
+    row), and optional position-sorted output."""
+    import torch
+    _require(q, torch.bfloat16, "q")
+    dev = q.device
+    _require(kcache, torch.bfloat16, "kcache", dev)
+    _require(w, torch.float32, "w", dev)
+    batch, heads, d = q.shape
+    if kcache.dim() == 2:
+        S, stride = kcache.shape[0], 0
+    elif kcache.dim() == 3 and kcache.shape[0] == batch:
+        S, stride = kcache.shape[1], kcache.shape[1]
+    else:
+        raise ValueError("kcache must be [S, d] or [batch, S, d]")
+    if kcache.shape[-1] != d or tuple(w.shape) != (batch, heads):
+        raise ValueError("shape mismatch between q, kcache and w")
+    if valid_len is not None:
+        _require(valid_len, torch.int32, "valid_len", dev)
+    if out_idx is None:
+        out_idx = torch.empty((batch, k), dtype=torch.int32, device=dev)
+    _require(out_idx, torch.int32, "out_idx", dev)
+    if return_score and out_score is None:
+        out_score = torch.empty((batch, k), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        rc = load().ds_indexer_topk_ex(_ptr(q), _ptr(kcache), int(stride), _ptr(w), batch, heads, d, S,
+                                       _ptr(valid_len), k, int(bool(sorted_index)), _ptr(out_idx),
+                                       _ptr(out_score) if return_score else None, _stream_ptr(stream))
+    _check(rc, "ds_indexer_topk_ex")
+    return out_idx, (out_score if return_score else None)

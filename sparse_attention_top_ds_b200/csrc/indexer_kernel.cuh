@@ -22,6 +22,8 @@
 //    shared memory) and the head sum are a register loop with no shuffles.
 //  * Positions at or past the group's largest valid_len are neither loaded
 //    nor multiplied.
+//  * The key tensor map is 3-D (channels, positions, caches): one cache for
+//    every row, or one per row (then a group is one row and reads cache t).
 #pragma once
 
 #include <cuda.h>
@@ -39,6 +41,7 @@ struct ScoreParams {
   int B, H, S;
   int tiles_per_cta;        // 128-position tiles per CTA
   int ctas_per_group;       // CTAs sharing one group of NT rows
+  int key_per_row;          // 1: row t reads key cache t (then NT == 1); 0: one cache for every row
 };
 
 template <int NT, int HP, int STAGES>
@@ -105,6 +108,7 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
     }
   }
   const int act_hi = min(tile_hi, (maxvl + 127) / 128);
+  const int kcache = p.key_per_row ? t0 : 0;  // the key cache of this group (its one row, with per-row caches)
   const int nact = max(0, act_hi - tile_lo);  // tiles that need the tensor cores
 
   if (threadIdx.x == 0) {
@@ -126,8 +130,8 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
       for (int i = 0; i < min(nact, STAGES); ++i) {
         const int pos0 = (tile_lo + i) * 128;
         mbar_arrive_expect_tx(BAR(C::kBarKFull + i), C::kStage);
-        tma_load_2d(sbase + C::kOffK + i * C::kStage, &tm_k, 0, pos0, BAR(C::kBarKFull + i));
-        tma_load_2d(sbase + C::kOffK + i * C::kStage + C::kKHalf, &tm_k, 64, pos0, BAR(C::kBarKFull + i));
+        tma_load_3d(sbase + C::kOffK + i * C::kStage, &tm_k, 0, pos0, kcache, BAR(C::kBarKFull + i));
+        tma_load_3d(sbase + C::kOffK + i * C::kStage + C::kKHalf, &tm_k, 64, pos0, kcache, BAR(C::kBarKFull + i));
       }
     }
   }
@@ -153,8 +157,8 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
         if (!mbar_wait_bounded(BAR(C::kBarKEmpty + s), (r & 1) ^ 1, p.status)) break;
         const int pos0 = (tile_lo + i) * 128;
         mbar_arrive_expect_tx(BAR(C::kBarKFull + s), C::kStage);
-        tma_load_2d(sbase + C::kOffK + s * C::kStage, &tm_k, 0, pos0, BAR(C::kBarKFull + s));
-        tma_load_2d(sbase + C::kOffK + s * C::kStage + C::kKHalf, &tm_k, 64, pos0, BAR(C::kBarKFull + s));
+        tma_load_3d(sbase + C::kOffK + s * C::kStage, &tm_k, 0, pos0, kcache, BAR(C::kBarKFull + s));
+        tma_load_3d(sbase + C::kOffK + s * C::kStage + C::kKHalf, &tm_k, 64, pos0, kcache, BAR(C::kBarKFull + s));
       }
     }
   } else if (warp == 1) {

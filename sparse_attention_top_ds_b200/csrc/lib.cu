@@ -310,6 +310,8 @@ static cudaError_t indexer_setup() {
   if (e == cudaSuccess) e = set_score_smem<4, 64, 4>();
   if (e == cudaSuccess) e = set_score_smem<8, 32, 4>();
   if (e == cudaSuccess) e = set_score_smem<8, 16, 4>();
+  if (e == cudaSuccess) e = set_score_smem<1, 32, 4>();
+  if (e == cudaSuccess) e = set_score_smem<1, 16, 4>();
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(indexer_topk_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              DecodeSmem::kBytes);
@@ -385,12 +387,27 @@ static bool encode_maps(const void* q, const void* kc, int B, int H, int S, int 
   return r == CUDA_SUCCESS;
 }
 
+// Keys viewed as (128 channels, S positions, nk caches), caches kstride rows
+// apart, in boxes of (64, 128, 1).
+static bool encode_kmap3(const void* kc, int S, int nk, long long kstride, CUtensorMap* tk) {
+  cuuint64_t dims[3] = {128, (cuuint64_t)S, (cuuint64_t)nk};
+  cuuint64_t str[2] = {256, (cuuint64_t)(kstride > 0 ? kstride : S) * 256};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t one[3] = {1, 1, 1};
+  return g_encode(tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kc), dims, str, box, one,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int NT, int HP, int ST>
 static int launch_score(const void* q, const void* kc, const float* w, int B, int H, int S, const int32_t* vl,
-                        float* out, cudaStream_t st, DeviceState* s) {
+                        float* out, long long kstride, cudaStream_t st, DeviceState* s) {
   using Cfg = ScoreCfg<NT, HP, ST>;
   CUtensorMap tq, tk;
   if (!encode_maps(q, kc, B, H, S, HP, NT, &tq, &tk)) return DS_ERR_ARG;
+  const bool per_row = kstride > 0;
+  if (per_row && NT != 1) return DS_ERR_ARG;
+  if (!encode_kmap3(kc, S, per_row ? B : 1, kstride, &tk)) return DS_ERR_ARG;
   const int ntiles = (S + 127) / 128;
   const int groups = (B + NT - 1) / NT;
   // spread one group's tiles over several CTAs only while there are fewer
@@ -409,6 +426,7 @@ static int launch_score(const void* q, const void* kc, const float* w, int B, in
   p.S = S;
   p.tiles_per_cta = (int)tpc;
   p.ctas_per_group = cpg;
+  p.key_per_row = per_row ? 1 : 0;
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)(groups * cpg), 1, 1);
@@ -423,18 +441,24 @@ static int launch_score(const void* q, const void* kc, const float* w, int B, in
   return e == cudaSuccess ? DS_OK : DS_ERR_CUDA;
 }
 
+// kstride: rows from one row's key cache to the next (0: one cache for every row).
 static int score_enqueue(const void* q, const void* kc, const float* w, int B, int H, int S, const int32_t* vl,
-                         float* out, cudaStream_t st, DeviceState* s) {
+                         float* out, cudaStream_t st, DeviceState* s, long long kstride = 0) {
+  if (kstride > 0) {  // a cache per row: one row per CTA group
+    if (H > 32) return launch_score<1, 64, 4>(q, kc, w, B, H, S, vl, out, kstride, st, s);
+    if (H > 16) return launch_score<1, 32, 4>(q, kc, w, B, H, S, vl, out, kstride, st, s);
+    return launch_score<1, 16, 4>(q, kc, w, B, H, S, vl, out, kstride, st, s);
+  }
   if (H > 32) {
-    if (B == 1) return launch_score<1, 64, 4>(q, kc, w, B, H, S, vl, out, st, s);
-    if (B == 2) return launch_score<2, 64, 4>(q, kc, w, B, H, S, vl, out, st, s);
+    if (B == 1) return launch_score<1, 64, 4>(q, kc, w, B, H, S, vl, out, 0, st, s);
+    if (B == 2) return launch_score<2, 64, 4>(q, kc, w, B, H, S, vl, out, 0, st, s);
     // 5..8 rows: two rows per CTA (measured faster than eight per CTA, whose
     // 128 KiB query tile every CTA must load)
-    if (B <= 4 || B > 8) return launch_score<4, 64, 4>(q, kc, w, B, H, S, vl, out, st, s);
-    return launch_score<2, 64, 4>(q, kc, w, B, H, S, vl, out, st, s);
+    if (B <= 4 || B > 8) return launch_score<4, 64, 4>(q, kc, w, B, H, S, vl, out, 0, st, s);
+    return launch_score<2, 64, 4>(q, kc, w, B, H, S, vl, out, 0, st, s);
   }
-  if (H > 16) return launch_score<8, 32, 4>(q, kc, w, B, H, S, vl, out, st, s);
-  return launch_score<8, 16, 4>(q, kc, w, B, H, S, vl, out, st, s);
+  if (H > 16) return launch_score<8, 32, 4>(q, kc, w, B, H, S, vl, out, 0, st, s);
+  return launch_score<8, 16, 4>(q, kc, w, B, H, S, vl, out, 0, st, s);
 }
 
 // ---- fused decode (score + top-k in one cooperative launch)
@@ -1001,4 +1025,24 @@ extern "C" int ds_indexer_qproj(const void* x, const void* wq, const void* ww, i
   cfg.attrs = attr;
   cfg.numAttrs = pdl_on() ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, indexer_qproj_kernel, p) == cudaSuccess ? DS_OK : DS_ERR_CUDA;
+}
+
+extern "C" int ds_indexer_topk_ex(const void* q, const void* kcache, int64_t kcache_batch_stride, const float* w,
+                                  int batch, int heads, int d, int S, const int32_t* valid_len, int k,
+                                  int sorted_index, int32_t* out_idx, float* out_score, void* stream) {
+  int rc = indexer_check(q, kcache, w, batch, heads, d, S);
+  if (rc != DS_OK) return rc;
+  if (!out_idx || k <= 0 || k > DS_MAX_K || S > kMaxRowElems) return DS_ERR_ARG;
+  if (kcache_batch_stride < 0 || (kcache_batch_stride > 0 && kcache_batch_stride < S)) return DS_ERR_ARG;
+  if (sorted_index != 0 && sorted_index != 1) return DS_ERR_ARG;
+  DeviceState* s = nullptr;
+  rc = device_state(&s);
+  if (rc != DS_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* scores = static_cast<float*>(get_scratch(s, (size_t)batch * (size_t)S * sizeof(float)));
+  if (!scores) return DS_ERR_NOMEM;
+  rc = score_enqueue(q, kcache, w, batch, heads, S, valid_len, scores, st, s, (long long)kcache_batch_stride);
+  if (rc != DS_OK) return rc;
+  return topk_enqueue(scores, batch, S, k, DS_F32, valid_len, out_idx, out_score, out_score != nullptr, sorted_index,
+                      st, s);
 }

@@ -29,8 +29,8 @@ def declared_entry_points():
 
 def test_header_declares_the_boundary():
     names = declared_entry_points()
-    for n in ("ds_topk", "ds_indexer_score", "ds_indexer_topk", "ds_indexer_qproj", "ds_sparse_attention",
-              "ds_get_device_status", "ds_strerror", "ds_release"):
+    for n in ("ds_topk", "ds_indexer_score", "ds_indexer_topk", "ds_indexer_topk_ex", "ds_indexer_qproj",
+              "ds_sparse_attention", "ds_get_device_status", "ds_strerror", "ds_release"):
         assert n in names
 
 
@@ -112,6 +112,28 @@ def test_attention_argument_errors_need_no_gpu(lib):
     assert call(out=vp(0x100002)) == -1
     assert call(W=8, win=vp(0x100008)) == -1
     assert call(lse=vp(0x100002)) == -1
+
+
+def test_indexer_topk_ex_argument_errors_need_no_gpu(lib):
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    f = lib.ds_indexer_topk_ex
+    f.restype = i32
+    f.argtypes = [vp, vp, ctypes.c_int64, vp, i32, i32, i32, i32, vp, i32, i32, vp, vp, vp]
+    a = vp(0x100000)
+
+    def call(stride=0, S=1000, k=100, sorted_index=0, d=128, H=64, q=a, idx=a):
+        return f(q, a, stride, a, 2, H, d, S, None, k, sorted_index, idx, None, None)
+
+    assert call(stride=-1) == -1
+    assert call(stride=999) == -1          # shorter than a cache
+    assert call(sorted_index=2) == -1
+    assert call(k=0) == -1
+    assert call(k=2049) == -1
+    assert call(d=64) == -1
+    assert call(H=65) == -1
+    assert call(q=None) == -1
+    assert call(idx=None) == -1
+    assert call(S=(1 << 24) + 1, stride=0) == -1
 
 
 def test_qproj_argument_errors_need_no_gpu(lib):

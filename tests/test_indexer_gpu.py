@@ -329,3 +329,90 @@ def test_rowcluster_graph_replay(cuda_device, rowcluster):
         assert ds.ds_get_device_status() == ds.DS_OK
         for o in outs:
             check_selection(q, kc, w, vl, 512, o.cpu().numpy(), None)
+
+
+# ---------------------------------------------------------------- per-row key caches, sorted output
+
+def _per_row_case(seed, B, H, S):
+    g = np.random.default_rng(seed)
+    q, _, w = inputs.indexer_factors(seed=seed, batch=B, n=S, heads=H, d=128)
+    kc3 = np.stack([inputs.indexer_factors(seed=seed + 100 + b, batch=1, n=S, heads=1, d=128)[1] for b in range(B)])
+    vl = g.integers(1, S, size=B, endpoint=True).astype(np.int32)
+    return q, kc3, w, vl
+
+
+@pytest.mark.parametrize("B,H,S,k", [(4, 64, 2000, 300), (3, 32, 700, 128), (3, 16, 700, 64), (2, 8, 500, 33),
+                                     (1, 64, 4096, 2048)])
+def test_per_row_key_caches(cuda_device, B, H, S, k):
+    q, kc3, w, vl = _per_row_case(40 + H, B, H, S)
+    qd, kd, wd, vd = dev_inputs(q, kc3, w, vl)
+    idx, score = ds.ds_indexer_topk_ex(qd, kd, wd, k, valid_len=vd, return_score=True)
+    torch.cuda.synchronize()
+    assert ds.ds_get_device_status() == ds.DS_OK
+    check_selection(q, kc3, w, vl, k, idx.cpu().numpy(), score.cpu().numpy())
+
+
+def test_per_row_exact_arithmetic_selects_exactly(cuda_device):
+    # small integer q and keys, power-of-two w: every float32 sum is exact, so the
+    # selected sets equal the oracle's (ties to the lower position)
+    g = np.random.default_rng(77)
+    B, H, S, k = 3, 64, 900, 100
+    q = inputs.f32_to_bf16_bits(g.integers(-2, 3, (B, H, 128)).astype(np.float32))
+    kc3 = inputs.f32_to_bf16_bits(g.integers(-2, 3, (B, S, 128)).astype(np.float32))
+    w = (2.0 ** g.integers(-3, 3, (B, H))).astype(np.float32)
+    vl = np.array([900, 450, 1], dtype=np.int32)
+    qd, kd, wd, vd = dev_inputs(q, kc3, w, vl)
+    idx, _ = ds.ds_indexer_topk_ex(qd, kd, wd, k, valid_len=vd)
+    torch.cuda.synchronize()
+    ref, _ = oracle.indexer_topk(q, kc3, w, k, vl)
+    got = idx.cpu().numpy()
+    for t in range(B):
+        m = int((ref[t] >= 0).sum())
+        assert sorted(got[t, :m].tolist()) == sorted(ref[t, :m].tolist())
+        assert np.all(got[t, m:] == -1)
+
+
+def test_ex_with_one_cache_matches_ds_indexer_topk(cuda_device):
+    q, kc, w, vl = inputs.decode(seed=51, batch=8, S=8192, vl_lo=1000, vl_hi=8192)
+    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
+    a, _ = ds.ds_indexer_topk(qd, kd, wd, 1024, valid_len=vd)
+    b, _ = ds.ds_indexer_topk_ex(qd, kd, wd, 1024, valid_len=vd)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.sort(a, dim=1).values, torch.sort(b, dim=1).values)
+
+
+@pytest.mark.parametrize("per_row", [False, True], ids=["one-cache", "per-row"])
+def test_sorted_index_in_the_fused_path(cuda_device, per_row):
+    if per_row:
+        q, kc, w, vl = _per_row_case(61, 4, 64, 3000)
+    else:
+        q, kc, w, vl = inputs.decode(seed=62, batch=4, S=3000, vl_lo=100, vl_hi=3000)
+    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
+    u, su = ds.ds_indexer_topk_ex(qd, kd, wd, 512, valid_len=vd, return_score=True)
+    s, ss = ds.ds_indexer_topk_ex(qd, kd, wd, 512, valid_len=vd, sorted_index=True, return_score=True)
+    torch.cuda.synchronize()
+    u, su, s, ss = u.cpu().numpy(), su.cpu().numpy(), s.cpu().numpy(), ss.cpu().numpy()
+    for t in range(4):
+        m = int((u[t] >= 0).sum())
+        assert np.all(np.diff(s[t, :m]) > 0), "not in ascending position order"
+        assert sorted(u[t, :m].tolist()) == s[t, :m].tolist()
+        order = np.argsort(u[t, :m])
+        assert np.array_equal(su[t, :m][order], ss[t, :m]), "scores do not follow their positions"
+    check_selection(q, kc, w, vl, 512, s, ss)
+
+
+def test_cache_stride_larger_than_S(cuda_device):
+    # caches padded with 37 extra rows each, addressed through the stride
+    B, H, S, k = 3, 64, 1200, 200
+    q, kc3, w, vl = _per_row_case(71, B, H, S)
+    padded = np.zeros((B, S + 37, 128), dtype=np.uint16)
+    padded[:, :S] = kc3
+    padded[:, S:] = inputs.f32_to_bf16_bits(np.full((B, 37, 128), 30.0, dtype=np.float32))  # would win if read
+    qd, kd, wd, vd = dev_inputs(q, padded, w, vl)
+    idx = torch.empty((B, k), dtype=torch.int32, device=cuda_device)
+    from sparse_attention_top_ds_b200._native import load, _ptr, _stream_ptr
+    rc = load().ds_indexer_topk_ex(_ptr(qd), _ptr(kd), S + 37, _ptr(wd), B, H, 128, S, _ptr(vd), k, 0,
+                                   _ptr(idx), None, _stream_ptr(None))
+    assert rc == ds.DS_OK
+    torch.cuda.synchronize()
+    check_selection(q, kc3, w, vl, k, idx.cpu().numpy(), None)
