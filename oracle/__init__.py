@@ -28,9 +28,14 @@ selection step computes, in float64:
                     "How the algorithm works", steps table, row 2) followed by
                     the same top-k.
 
+* ``compress``   -- the compressor's 4:1 fold as a gated weighted sum (NKI pull
+                    request, steps table row 1).  PARITY UNPINNED: the pages do
+                    not give the gate, so the function follows a stated reading.
+
 Every function is pinned by the ``-m "not gpu"`` tests in ``tests/test_oracle_*``
 against brute force, closed forms, hand-worked examples under ``tests/golden``
-and invariants; no function here is "parity unpinned".
+and invariants.  ``compress_fold`` alone is "parity unpinned": its pins check
+the stated reading of the gate, which no page fixes.
 """
 
 from .encoding import decode_bf16, decode_f32, NEG_INF_BF16, NEG_INF_F32
@@ -38,8 +43,9 @@ from .topk import topk_rows, topk_row
 from .indexer import indexer_scores, indexer_topk
 from .attention import sparse_attention
 from .qproj import qproj, round_bf16
+from .compress import compress_fold
 
 __all__ = [
     "decode_bf16", "decode_f32", "NEG_INF_BF16", "NEG_INF_F32",
-    "topk_rows", "topk_row", "indexer_scores", "indexer_topk", "sparse_attention", "qproj", "round_bf16",
+    "topk_rows", "topk_row", "indexer_scores", "indexer_topk", "sparse_attention", "qproj", "round_bf16", "compress_fold",
 ]
