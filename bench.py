@@ -222,6 +222,24 @@ def measure_qproj(ds, inputs, dev, stream, rank, hbm_gbs, calls, warmup=3):
     }
 
 
+def measure_compress(ds, inputs, dev, rank):
+    """The compressor's 4:1 fold of a decode step: 8 batch rows, 4 new rows of
+    the attention's width 512 each, folded into position 0 of a compressed
+    cache.  A few KiB per call: latency bound, so the number is µs per call
+    (CUDA-graph replays of 64 calls over 4 rotating input copies)."""
+    import torch
+    rows, gate = inputs.compress(seed=inputs.SEED_COMPRESS + rank, batch=8, D=512)
+    to = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    rs = [to(rows) for _ in range(4)]
+    gd = to(gate)
+    cache = torch.empty((8, 64, 512), dtype=torch.bfloat16, device=dev)
+    us = graph_time_us(lambda i: ds.ds_compress_fold(rs[i % 4], gd, out=cache[:, i % 64, :]), 64, reps=3)
+    (us,) = max_over_ranks([us], dev)
+    return {"workload": "8 batch rows x 4 rows x 512 bf16 -> 8 folded rows written into a [8, 64, 512] cache",
+            "us_per_call": round(us, 2), "bound": "latency",
+            "bytes_per_call": int(rows.nbytes + gate.nbytes + 8 * 512 * 2)}
+
+
 def run_attention_only(args):
     """`--only attention` / `--only qproj`: one beside-the-headline measurement
     alone (the commands the profiles of those kernels are taken with)."""
@@ -562,6 +580,7 @@ def run_ours(args):
 
     attention = measure_attention(ds, inputs, dev, stream, rank, hbm_gbs, tflops, ATTN_CALLS)
     qproj = measure_qproj(ds, inputs, dev, stream, rank, hbm_gbs, ATTN_CALLS)
+    compress = measure_compress(ds, inputs, dev, rank)
 
     traffic = None
     prof = os.path.join(ROOT, "profiles", "topk_traffic.json")
@@ -607,6 +626,7 @@ def run_ours(args):
                         "bf16_peak_tflops": tflops_sus, "peak_kind": "sustained"},
             "sparse_attention": attention,
             "qproj": qproj,
+            "compress_fold": compress,
             "roofline": {"bound": "hbm", "achieved": round(per_launch_gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
                          "frac": round(per_launch_gbs / hbm_gbs, 4), "traffic": traffic,
                          "kernel": TOPK_KERNEL, "peak_source": peak_src},

@@ -2,7 +2,7 @@
  * ds_topk.h -- C ABI of libdstopk.so, the selection step of DeepSeek-style
  * sparse attention on B200 (sm_100a).
  *
- * Four operations, as described on the pages this library follows:
+ * Five operations, as described on the pages this library follows:
  *
  *  - Row-wise top-k of given scores (DeepSelect hub page, use-case paragraphs:
  *    pick the top-k positions of every score row; bfloat16 rows for the
@@ -15,6 +15,9 @@
  *        score[t,s] = sum_h w[t,h] * max(0, q[t,h,:] . k[s,:])
  *    over a 128-channel bfloat16 key cache shared by all rows, then the k
  *    highest-scoring positions of each row.
+ *
+ *  - The compressor's 4:1 fold of new rows into the compressed caches (steps
+ *    table row 1; the gate is a stated reading, the pages give none).
  *
  *  - The indexer query projection that produces the scorer's queries and
  *    per-head weights (the same pull request, steps table row 2).
@@ -222,6 +225,33 @@ int ds_indexer_topk_noalloc(const void* q, const void* kcache, const float* w,
  */
 int ds_indexer_qproj(const void* x, const void* wq, const void* ww, int T, int d_in, int heads, int d,
                      void* q_out, float* w_out, void* stream);
+
+/*
+ * ds_compress_fold -- the compressor's 4:1 fold: 4 rows into 1 by a gated
+ * weighted sum.
+ *   (NKI pull request "Add DeepSeek-V4 CSA attention kernels", "How the
+ *    algorithm works", steps table row 1: the compressor folds 4 tokens into
+ *    1 with a gated weighted sum, once every 4 decode steps.)
+ *
+ * The pages do not give the gate.  The reading implemented: per-token scores
+ * s_i = gate . x_i (float32 from the bf16 products), weights
+ * a = softmax(s_0..s_3), folded row = sum_i a_i x_i, rounded to bfloat16.
+ *
+ * rows     device bfloat16: batch row b's 4 rows of D elements start
+ *          rows_batch_stride * b elements after rows, each D after the last
+ *          (a [batch, 4, D] array: stride 4 * D); 16-byte aligned.
+ * batch    >= 1.   D: a multiple of 8, 8 <= D <= 4096.
+ * rows_batch_stride  >= 4 * D, a multiple of 8 (elements).
+ * gate     device bfloat16 [D]; 16-byte aligned.
+ * out      device bfloat16: batch row b's folded row at out +
+ *          out_batch_stride * b (for instance position j of a [batch, T_c, D]
+ *          cache: out = cache + j * D, out_batch_stride = T_c * D);
+ *          16-byte aligned.
+ * out_batch_stride  >= D, a multiple of 8 (elements).
+ * Returns DS_OK, DS_ERR_ARG, DS_ERR_UNSUPPORTED or DS_ERR_CUDA.
+ */
+int ds_compress_fold(const void* rows, int batch, int D, int64_t rows_batch_stride, const void* gate,
+                     void* out, int64_t out_batch_stride, void* stream);
 
 /*
  * ds_sparse_attention -- multi-query decode attention over the selected

@@ -16,7 +16,7 @@ from ._native import (  # noqa: F401
     DS_F32, DS_BF16, DS_OK, DS_ERR_ARG, DS_ERR_CUDA, DS_ERR_TIMEOUT, DS_ERR_UNSUPPORTED,
     DS_ERR_NOMEM, DS_MAX_K, DS_INDEXER_DIM, DS_INDEXER_MAX_HEADS, DS_ATTN_MAX_DIM, DS_ATTN_MAX_WINDOW,
     DS_ATTN_MAX_HEADS, DsError,
-    ds_topk, ds_indexer_score, ds_indexer_topk, ds_indexer_topk_ex, ds_indexer_qproj, ds_sparse_attention, ds_get_device_status,
+    ds_topk, ds_indexer_score, ds_indexer_topk, ds_indexer_topk_ex, ds_indexer_qproj, ds_compress_fold, ds_sparse_attention, ds_get_device_status,
     ds_release,
     strerror, load, lib_path,
 )

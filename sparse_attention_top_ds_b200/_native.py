@@ -65,6 +65,8 @@ def load():
     lib.ds_sparse_attention.restype = i32
     lib.ds_indexer_topk_ex.argtypes = [vp, vp, ctypes.c_int64, vp, i32, i32, i32, i32, i32p, i32, i32, vp, vp, vp]
     lib.ds_indexer_topk_ex.restype = i32
+    lib.ds_compress_fold.argtypes = [vp, i32, i32, ctypes.c_int64, vp, vp, ctypes.c_int64, vp]
+    lib.ds_compress_fold.restype = i32
     lib.ds_indexer_qproj.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp]
     lib.ds_indexer_qproj.restype = i32
     lib.ds_get_device_status.argtypes = [vp]
@@ -360,3 +362,31 @@ def ds_indexer_topk_ex(q, kcache, w, k, valid_len=None, sorted_index=False, retu
                                        _ptr(out_score) if return_score else None, _stream_ptr(stream))
     _check(rc, "ds_indexer_topk_ex")
     return out_idx, (out_score if return_score else None)
+
+
+def ds_compress_fold(rows, gate, out=None, stream=None):
+    """Fold each batch row's 4 rows into 1 (gated weighted sum).
+
+    rows bf16 [batch, 4, D] (any batch stride, rows contiguous within a batch
+    row); gate bf16 [D]; out bf16 [batch, D] or a strided [batch, D] view (for
+    instance cache[:, j, :]).  Returns out.
+    """
+    import torch
+    if not isinstance(rows, torch.Tensor) or rows.dtype != torch.bfloat16 or not rows.is_cuda:
+        raise TypeError("rows must be a CUDA bfloat16 tensor")
+    if rows.dim() != 3 or rows.shape[1] != 4 or rows.stride(2) != 1 or rows.stride(1) != rows.shape[2]:
+        raise ValueError("rows must be [batch, 4, D] with contiguous rows")
+    dev = rows.device
+    batch, _, D = rows.shape
+    _require(gate, torch.bfloat16, "gate", dev)
+    if gate.numel() != D:
+        raise ValueError("gate must hold D elements")
+    if out is None:
+        out = torch.empty((batch, D), dtype=torch.bfloat16, device=dev)
+    if out.dtype != torch.bfloat16 or out.device != dev or out.dim() != 2 or out.stride(1) != 1 or out.shape[1] != D:
+        raise ValueError("out must be a [batch, D] bfloat16 view with contiguous rows")
+    with torch.cuda.device(dev):
+        rc = load().ds_compress_fold(_ptr(rows), batch, D, rows.stride(0), _ptr(gate), _ptr(out), out.stride(0),
+                                     _stream_ptr(stream))
+    _check(rc, "ds_compress_fold")
+    return out

@@ -20,6 +20,7 @@
 #include "rowcluster_kernel.cuh"
 #include "attention_kernel.cuh"
 #include "qproj_kernel.cuh"
+#include "compress_kernel.cuh"
 
 namespace dstopk {
 
@@ -1045,4 +1046,35 @@ extern "C" int ds_indexer_topk_ex(const void* q, const void* kcache, int64_t kca
   if (rc != DS_OK) return rc;
   return topk_enqueue(scores, batch, S, k, DS_F32, valid_len, out_idx, out_score, out_score != nullptr, sorted_index,
                       st, s);
+}
+
+extern "C" int ds_compress_fold(const void* rows, int batch, int D, int64_t rows_batch_stride, const void* gate,
+                                void* out, int64_t out_batch_stride, void* stream) {
+  auto misaligned = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; };
+  if (!rows || !gate || !out || batch <= 0 || batch > (1 << 24)) return DS_ERR_ARG;
+  if (D < 8 || D > kCfMaxD || D % 8 != 0) return DS_ERR_ARG;
+  if (rows_batch_stride < 4LL * D || rows_batch_stride % 8 != 0) return DS_ERR_ARG;
+  if (out_batch_stride < (int64_t)D || out_batch_stride % 8 != 0) return DS_ERR_ARG;
+  if (misaligned(rows, 16) || misaligned(gate, 16) || misaligned(out, 16)) return DS_ERR_ARG;
+  DeviceState* s = nullptr;
+  const int rc = device_state(&s);
+  if (rc != DS_OK) return rc;
+  CfParams p;
+  p.rows = static_cast<const uint16_t*>(rows);
+  p.gate = static_cast<const uint16_t*>(gate);
+  p.out = static_cast<uint16_t*>(out);
+  p.rows_bstride = (long long)rows_batch_stride;
+  p.out_bstride = (long long)out_batch_stride;
+  p.B = batch;
+  p.D = D;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)((batch + kCfWarps - 1) / kCfWarps), 1, 1);
+  cfg.blockDim = dim3(kCfWarps * 32, 1, 1);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  set_pdl(attr[0]);
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_on() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, compress_fold_kernel, p) == cudaSuccess ? DS_OK : DS_ERR_CUDA;
 }

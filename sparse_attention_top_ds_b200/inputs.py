@@ -40,6 +40,7 @@ SEED_DECODE = 1004
 SEED_PREFILL = 1005
 SEED_ATTENTION = 1006
 SEED_QPROJ = 1007
+SEED_COMPRESS = 1008
 
 
 def rng(seed):
@@ -192,3 +193,12 @@ def attention_slots(seed, batch=8, T=32768, k=1024, vl_lo=4096, vl_hi=32768):
         m = min(k, L)
         idx[b, :m] = g.choice(L, size=m, replace=False)
     return idx
+
+
+def compress(seed=SEED_COMPRESS, batch=8, D=512, gate_scale=1.0):
+    """Compressor inputs: (rows [batch, 4, D], gate [D]) bfloat16 patterns of
+    rows ~ N(0, 1) and gate ~ N(0, gate_scale^2 / D) (gate scores ~ N(0, gate_scale^2))."""
+    g = rng(seed)
+    rows = f32_to_bf16_bits(g.standard_normal((batch, 4, D), dtype=np.float32))
+    gate = f32_to_bf16_bits(g.standard_normal(D, dtype=np.float32) * np.float32(gate_scale / np.sqrt(D)))
+    return rows, gate

@@ -30,7 +30,7 @@ def declared_entry_points():
 def test_header_declares_the_boundary():
     names = declared_entry_points()
     for n in ("ds_topk", "ds_indexer_score", "ds_indexer_topk", "ds_indexer_topk_ex", "ds_indexer_qproj",
-              "ds_sparse_attention", "ds_get_device_status", "ds_strerror", "ds_release"):
+              "ds_compress_fold", "ds_sparse_attention", "ds_get_device_status", "ds_strerror", "ds_release"):
         assert n in names
 
 
@@ -134,6 +134,30 @@ def test_indexer_topk_ex_argument_errors_need_no_gpu(lib):
     assert call(q=None) == -1
     assert call(idx=None) == -1
     assert call(S=(1 << 24) + 1, stride=0) == -1
+
+
+def test_compress_argument_errors_need_no_gpu(lib):
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    f = lib.ds_compress_fold
+    f.restype = i32
+    f.argtypes = [vp, i32, i32, ctypes.c_int64, vp, vp, ctypes.c_int64, vp]
+    a = vp(0x100000)
+
+    def call(rows=a, B=8, D=512, rs=2048, gate=a, out=a, os_=512):
+        return f(rows, B, D, rs, gate, out, os_, None)
+
+    assert call(rows=None) == -1
+    assert call(gate=None) == -1
+    assert call(out=None) == -1
+    assert call(B=0) == -1
+    assert call(D=4) == -1
+    assert call(D=4104, rs=4 * 4104, os_=4104) == -1
+    assert call(D=100) == -1              # not a multiple of 8
+    assert call(rs=2047) == -1            # shorter than 4 rows
+    assert call(rs=2052) == -1            # not a multiple of 8
+    assert call(os_=511) == -1
+    assert call(rows=vp(0x100008)) == -1  # 16-byte alignment
+    assert call(out=vp(0x100004)) == -1
 
 
 def test_qproj_argument_errors_need_no_gpu(lib):
