@@ -22,8 +22,11 @@
 //    shared memory) and the head sum are a register loop with no shuffles.
 //  * Positions at or past the group's largest valid_len are neither loaded
 //    nor multiplied.
-//  * The key tensor map is 3-D (channels, positions, caches): one cache for
-//    every row, or one per row (then a group is one row and reads cache t).
+//  * The key tensor map is 4-D (64 channels, positions, 2 channel halves,
+//    caches): one TMA copy brings a whole 128-position tile (32 KiB), its two
+//    64-channel halves one after the other as the MMA reads them.  There is one
+//    cache for every row, or one per row (then a group is one row and reads
+//    cache t).
 #pragma once
 
 #include <cuda.h>
@@ -130,8 +133,7 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
       for (int i = 0; i < min(nact, STAGES); ++i) {
         const int pos0 = (tile_lo + i) * 128;
         mbar_arrive_expect_tx(BAR(C::kBarKFull + i), C::kStage);
-        tma_load_3d(sbase + C::kOffK + i * C::kStage, &tm_k, 0, pos0, kcache, BAR(C::kBarKFull + i));
-        tma_load_3d(sbase + C::kOffK + i * C::kStage + C::kKHalf, &tm_k, 64, pos0, kcache, BAR(C::kBarKFull + i));
+        tma_load_4d(sbase + C::kOffK + i * C::kStage, &tm_k, 0, pos0, 0, kcache, BAR(C::kBarKFull + i));
       }
     }
   }
@@ -157,8 +159,7 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
         if (!mbar_wait_bounded(BAR(C::kBarKEmpty + s), (r & 1) ^ 1, p.status)) break;
         const int pos0 = (tile_lo + i) * 128;
         mbar_arrive_expect_tx(BAR(C::kBarKFull + s), C::kStage);
-        tma_load_3d(sbase + C::kOffK + s * C::kStage, &tm_k, 0, pos0, kcache, BAR(C::kBarKFull + s));
-        tma_load_3d(sbase + C::kOffK + s * C::kStage + C::kKHalf, &tm_k, 64, pos0, kcache, BAR(C::kBarKFull + s));
+        tma_load_4d(sbase + C::kOffK + s * C::kStage, &tm_k, 0, pos0, 0, kcache, BAR(C::kBarKFull + s));
       }
     }
   } else if (warp == 1) {

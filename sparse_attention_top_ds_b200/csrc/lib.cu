@@ -388,14 +388,15 @@ static bool encode_maps(const void* q, const void* kc, int B, int H, int S, int 
   return r == CUDA_SUCCESS;
 }
 
-// Keys viewed as (128 channels, S positions, nk caches), caches kstride rows
-// apart, in boxes of (64, 128, 1).
+// Keys viewed as (64 channels, S positions, 2 channel halves, nk caches),
+// caches kstride rows apart, in boxes of (64, 128, 2, 1): one copy is a whole
+// 128-position tile, its two 64-channel halves one after the other.
 static bool encode_kmap3(const void* kc, int S, int nk, long long kstride, CUtensorMap* tk) {
-  cuuint64_t dims[3] = {128, (cuuint64_t)S, (cuuint64_t)nk};
-  cuuint64_t str[2] = {256, (cuuint64_t)(kstride > 0 ? kstride : S) * 256};
-  cuuint32_t box[3] = {64, 128, 1};
-  cuuint32_t one[3] = {1, 1, 1};
-  return g_encode(tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kc), dims, str, box, one,
+  cuuint64_t dims[4] = {64, (cuuint64_t)S, 2, (cuuint64_t)nk};
+  cuuint64_t str[3] = {256, 128, (cuuint64_t)(kstride > 0 ? kstride : S) * 256};
+  cuuint32_t box[4] = {64, 128, 2, 1};
+  cuuint32_t one[4] = {1, 1, 1, 1};
+  return g_encode(tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(kc), dims, str, box, one,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -451,6 +452,13 @@ static int score_enqueue(const void* q, const void* kc, const float* w, int B, i
     return launch_score<1, 16, 4>(q, kc, w, B, H, S, vl, out, kstride, st, s);
   }
   if (H > 32) {
+    const char* force = getenv("DS_SCORE_ROWS");  // tuning sweeps only: rows per CTA group
+    if (force && B > 2) {
+      const int nt = atoi(force);
+      if (nt == 1) return launch_score<1, 64, 4>(q, kc, w, B, H, S, vl, out, 0, st, s);
+      if (nt == 2) return launch_score<2, 64, 4>(q, kc, w, B, H, S, vl, out, 0, st, s);
+      if (nt == 4) return launch_score<4, 64, 4>(q, kc, w, B, H, S, vl, out, 0, st, s);
+    }
     if (B == 1) return launch_score<1, 64, 4>(q, kc, w, B, H, S, vl, out, 0, st, s);
     if (B == 2) return launch_score<2, 64, 4>(q, kc, w, B, H, S, vl, out, 0, st, s);
     // 5..8 rows: two rows per CTA (measured faster than eight per CTA, whose
