@@ -20,7 +20,7 @@ For one new token of batch row b, with queries q[b, h, :] of every head h:
     lse[b,h] = m[h] + log(l[h])
 
 in float64 from the exact bfloat16 / float32 inputs.  Readings where the pages
-are silent (listed in the design doc):
+are silent:
   * every query head attends to the same gathered rows (multi-query: one KV
     head), and each row serves as both key and value;
   * the selected rows and the window rows form one softmax ("concatenate");

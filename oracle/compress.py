@@ -7,7 +7,7 @@ the compressor folds 4 tokens into 1 with a gated weighted sum, once every 4
 decode steps.  How the gate is computed is not given on any page, so this
 function states one reading -- the plainest one that fits "gated weighted
 sum" -- and its pins check the function against that reading's closed forms,
-not against the pages.  the design doc lists the reading.
+not against the pages.
 
 Reading: each of the 4 tokens x_i (rows of width D) gets one gate score
 s_i = g . x_i from a gate vector g of width D; the weights are

@@ -9,7 +9,7 @@ highest-scoring positions):
     score[t, s] = sum over heads h of  w[t, h] * max(0, sum over c of q[t,h,c] * k[s,c])
 
 for positions s < valid_len[t], in float64 from the exact bfloat16 / float32
-inputs.  Readings where the pages are silent (listed in the design doc):
+inputs.  Readings where the pages are silent:
   * the ReLU applies to each head's dot product, then the weight multiplies it,
     then the heads are summed (the order the steps table names them in);
   * there is no extra scale factor (any scale folds into w);

@@ -9,7 +9,7 @@ before the scoring launch):
     w[t, h]    = sum_i x[t, i] * Ww[h, i]                 (kept in float32)
 
 in float64 from the exact bfloat16 inputs.  Readings where the pages are
-silent (listed in DESIGN.md):
+silent:
   * the projection is a plain linear map of one input vector per token, with no
     bias, normalisation, rotation or quantisation (none is named);
   * the per-head weights w of the indexer score come from a second linear map of

@@ -14,7 +14,7 @@ for each row t, with L = min(valid_len[t], n):
      copied unchanged;
   5. slots m..k-1 are padding: index -1, value -inf.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   * ties go to the lower index;
   * -0.0 and +0.0 are equal (the index decides);
   * every NaN ranks above +inf and all NaNs are equal (the index decides);

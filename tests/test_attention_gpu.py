@@ -1,6 +1,7 @@
 """GPU parity of ds_sparse_attention with the float64 oracle.
 
-The bar (derived in the design doc from the arithmetic): per batch row,
+The bar, from the arithmetic (the softmax weights are rounded to bfloat16
+twice, at most 2^-8 relative each, and the output once more): per batch row,
 max |out - out_ref| <= 1e-2 * max |value of an attended row|, and
 |lse - lse_ref| <= 5e-3; -inf lse and zero output exactly where nothing is
 attended.  Inputs come from sparse_attention_top_ds_b200.inputs, expected

@@ -1,8 +1,8 @@
 """GPU parity of ds_indexer_qproj with the float64 oracle.
 
 Both kernels are covered: input widths that are a multiple of 64 run on the
-tensor cores (TMA + tcgen05), the others on the CUDA cores.  The bar (the design doc
-derives it): |q - q_ref| <= 2^-8 |q_ref| + 2^-18 sum_i |x_i w_i|
+tensor cores (TMA + tcgen05), the others on the CUDA cores.  The bar, from the
+arithmetic: |q - q_ref| <= 2^-8 |q_ref| + 2^-18 sum_i |x_i w_i|
 (one bfloat16 rounding plus float32 accumulation), |w - w_ref| <= 2^-18 sum_i |x_i w_i|;
 bit-exact (q = bf16(q_ref), w = w_ref) where every partial sum is exact in float32.
 """
