@@ -198,3 +198,14 @@ def test_graph_replay(cuda_device):
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), first.view(torch.int16))
     assert ds.ds_get_device_status() == ds.DS_OK
+
+
+def test_largest_slots_and_window(cuda_device):
+    """k = 2048 slots plus the largest window (4096 rows): 96 chunks of 64 rows
+    per batch row, so the weighted-sum kernel runs its 2-chunk stages with the
+    largest statistics block; d = 512, 160 heads (two head tiles)."""
+    a = inputs.attention(seed=14, batch=2, heads=160, d=512, T=6000, k=2048, W=4096, shared_cache=False,
+                         vl_lo=3000, vl_hi=6000, holes=0.02, win_len=[4096, 1234])
+    scale = 1.0 / math.sqrt(512)
+    out, lse = _run(a, cuda_device, scale)
+    _check(a, out, lse, scale)
