@@ -282,37 +282,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // writes 32 columns.
 constexpr int kPvWarps = 10;
 constexpr int kPvRescale = 256;  // rescaling threads (warps 1..8)
-constexpr int kPvStages = 2;
-template <int K>
+// K chunks per ring stage, S ring stages
+template <int K, int S>
 struct PvSmem {
   static constexpr int kStage = K * (kAttnTile + kRowTile);
   // ring | partner's columns (128 heads x 32 floats) | (max, sum) of every chunk
-  // of the row | mbarriers full[2], ready[2], empty[2], ml, done, recv | TMEM slot
-  __host__ __device__ static constexpr int recv_off() { return kPvStages * kStage; }
+  // of the row | mbarriers full[S], ready[S], empty[S], ml, done, recv | TMEM slot
+  __host__ __device__ static constexpr int recv_off() { return S * kStage; }
   __host__ __device__ static constexpr int ml_off() { return recv_off() + kAttnHeads * 32 * 4; }
   __host__ __device__ static constexpr int bar_off(int NS) { return ml_off() + NS * kAttnHeads * 8; }
-  __host__ __device__ static constexpr int slot_off(int NS) { return bar_off(NS) + (3 * kPvStages + 3) * 8; }
+  __host__ __device__ static constexpr int slot_off(int NS) { return bar_off(NS) + (3 * S + 3) * 8; }
   __host__ __device__ static constexpr int bytes(int NS) { return slot_off(NS) + 16 + 1024; }
 };
 
 // Columns [LO, LO + 32) of one head's accumulator, held as r[0..31]:
-// optionally add the partner's share from `recv`, round to bf16 and store.
+// optionally add the partner's share from `recv` (the head's 128 bytes, whose
+// 16-byte piece i sits at position i ^ sw), round to bf16 and store.
 template <bool ADD>
-__device__ __forceinline__ void pv_emit(const uint32_t (&r)[32], const float* recv, uint16_t* dst) {
+__device__ __forceinline__ void pv_emit(const uint32_t (&r)[32], const float* recv, int sw, uint16_t* dst) {
   uint4* d4 = reinterpret_cast<uint4*>(dst);
+  const float4* r4 = reinterpret_cast<const float4*>(recv);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
+    float a[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+    if (ADD) {
+      const float4 x = r4[(2 * q) ^ sw], y = r4[(2 * q + 1) ^ sw];
+      a[0] = x.x, a[1] = x.y, a[2] = x.z, a[3] = x.w, a[4] = y.x, a[5] = y.y, a[6] = y.z, a[7] = y.w;
+    }
     float v[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * q + e]) + (ADD ? recv[8 * q + e] : 0.0f);
+    for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * q + e]) + a[e];
     d4[q] = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
                        pack_bf16x2(v[6], v[7]));
   }
 }
 
-template <int K>
+template <int K, int S>
 __global__ void __launch_bounds__(kPvWarps * 32, 1) sparse_attn_pv_kernel(const AttnParams p) {
-  using L_ = PvSmem<K>;
+  using L_ = PvSmem<K, S>;
+  constexpr int kPvStages = S;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -465,22 +473,25 @@ __global__ void __launch_bounds__(kPvWarps * 32, 1) sparse_attn_pv_kernel(const 
     uint16_t* orow = p.out + ((size_t)b * p.H + hg) * p.D + (size_t)slice * kPvSlice + half * 32;
     if (G == 2) {
       if (half != g) {
-        // these 32 columns are finalised by the partner (CTA `half` of the pair)
+        // these 32 columns are finalised by the partner (CTA `half` of the pair);
+        // piece q goes to position q ^ (h % 8) of the head's 128 bytes, so that
+        // eight consecutive heads write (and later read) eight bank groups
         const uint32_t dst = dsmem_map(smem_u32(recv + h * 32), (uint32_t)half);
         const uint32_t rbar = dsmem_map(bar_recv, (uint32_t)half);
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::
-                           "r"(dst + 16u * q), "r"(r[4 * q]), "r"(r[4 * q + 1]), "r"(r[4 * q + 2]), "r"(r[4 * q + 3]),
+                           "r"(dst + 16u * (uint32_t)(q ^ (h & 7))), "r"(r[4 * q]), "r"(r[4 * q + 1]), "r"(r[4 * q + 2]),
+                       "r"(r[4 * q + 3]),
                        "r"(rbar)
                        : "memory");
       } else {
         if (h == 0) mbar_arrive_expect_tx(bar_recv, kAttnHeads * 32 * 4);  // 128 heads x 32 columns from the partner
         mbar_wait_bounded(bar_recv, 0, p.status);
-        if (hg < p.H) pv_emit<true>(r, recv + h * 32, orow);
+        if (hg < p.H) pv_emit<true>(r, recv + h * 32, h & 7, orow);
       }
     } else if (hg < p.H) {
-      pv_emit<false>(r, recv, orow);
+      pv_emit<false>(r, recv, 0, orow);
     }
     if (half == 0 && hg < p.H && slice == 0 && g == 0 && p.lse)
       p.lse[(size_t)b * p.H + hg] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;

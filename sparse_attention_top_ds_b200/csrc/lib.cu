@@ -291,6 +291,31 @@ static int topk_enqueue(const void* scores, int batch, int n, int k, int dtype, 
 
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+// Ring shapes of the weighted-sum kernel (K chunks per stage, S stages), in
+// order of preference: the first whose shared memory fits the row's chunk count
+// is launched.  Deeper rings of smaller stages (2 x 3, 1 x 4 .. 1 x 7) were no
+// faster on the decode workload: the stream is bound by each SM's copy rate.
+struct PvCfg {
+  int K, S;
+  void (*fn)(AttnParams);
+  int (*bytes)(int);
+};
+template <int K, int S>
+static int pv_bytes(int NS) {
+  return PvSmem<K, S>::bytes(NS);
+}
+#define DS_PV_CFG(k, s) {k, s, sparse_attn_pv_kernel<k, s>, pv_bytes<k, s>}
+static const PvCfg kPvCfg[] = {DS_PV_CFG(4, 2), DS_PV_CFG(3, 2), DS_PV_CFG(2, 2), DS_PV_CFG(1, 2)};
+#undef DS_PV_CFG
+static constexpr int kPvCfgs = (int)(sizeof(kPvCfg) / sizeof(kPvCfg[0]));
+
+static const PvCfg* pv_pick(int NS) {
+  const int lim = 227 * 1024;
+  for (int i = 0; i < kPvCfgs; ++i)
+    if (kPvCfg[i].bytes(NS) <= lim) return &kPvCfg[i];
+  return nullptr;
+}
+
 template <int NT, int HP, int ST>
 static cudaError_t set_score_smem() {
   return cudaFuncSetAttribute(indexer_score_kernel<NT, HP, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -327,14 +352,8 @@ static cudaError_t indexer_setup() {
                              kQpTok * kQpMaxIn * 2 + 8 * 32 * 33 * 4);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(indexer_qproj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, QtSmem::kBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(sparse_attn_pv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(sparse_attn_pv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(sparse_attn_pv_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(sparse_attn_pv_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  for (int i = 0; e == cudaSuccess && i < kPvCfgs; ++i)
+    e = cudaFuncSetAttribute(kPvCfg[i].fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   return e;
 }
 
@@ -726,18 +745,13 @@ static int attention_enqueue(const uint16_t* q, const uint16_t* kv, long long kv
     // chunks of a row split over a cluster pair while one CTA per column slice
     // would leave more than half of the SMs idle
     const int G = (NS > 1 && 2L * (D / kPvSlice) * HT * nb <= s->num_sms) ? 2 : 1;
-    // the most chunks per ring stage that the row's statistics leave room for
-    const int lim = 227 * 1024;
-    const int K = PvSmem<4>::bytes(NS) <= lim ? 4 : (PvSmem<3>::bytes(NS) <= lim ? 3 : (PvSmem<2>::bytes(NS) <= lim ? 2 : 1));
-    if (PvSmem<1>::bytes(NS) > lim) return DS_ERR_ARG;
+    const PvCfg* pc = pv_pick(NS);
+    if (!pc) return DS_ERR_ARG;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3((unsigned)(D / kPvSlice), (unsigned)G, (unsigned)(HT * nb));
     cfg.blockDim = dim3(kPvWarps * 32, 1, 1);
-    cfg.dynamicSmemBytes = (size_t)(K == 4   ? PvSmem<4>::bytes(NS)
-                                    : K == 3 ? PvSmem<3>::bytes(NS)
-                                    : K == 2 ? PvSmem<2>::bytes(NS)
-                                             : PvSmem<1>::bytes(NS));
+    cfg.dynamicSmemBytes = (size_t)pc->bytes(NS);
     cfg.stream = st;
     cudaLaunchAttribute pattr[2];
     int na = 0;
@@ -751,11 +765,7 @@ static int attention_enqueue(const uint16_t* q, const uint16_t* kv, long long kv
     }
     cfg.attrs = pattr;
     cfg.numAttrs = na;
-    const cudaError_t e = K == 4   ? cudaLaunchKernelEx(&cfg, sparse_attn_pv_kernel<4>, p)
-                          : K == 3 ? cudaLaunchKernelEx(&cfg, sparse_attn_pv_kernel<3>, p)
-                          : K == 2 ? cudaLaunchKernelEx(&cfg, sparse_attn_pv_kernel<2>, p)
-                                   : cudaLaunchKernelEx(&cfg, sparse_attn_pv_kernel<1>, p);
-    if (e != cudaSuccess) return DS_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, pc->fn, p) != cudaSuccess) return DS_ERR_CUDA;
   }
   return DS_OK;
 }
