@@ -99,6 +99,19 @@ def test_matches_oracle(case, cuda_device):
     _check(a, out, lse, scale)
 
 
+def test_repeated_slots(cuda_device):
+    # a row picked by several slots is attended once per slot; the repeats sit in
+    # other 64-row chunks than the first pick, and one row repeats 40 times
+    a = inputs.attention(seed=8, batch=2, heads=128, d=512, T=3000, k=400, W=64, shared_cache=False,
+                         vl_lo=1000, vl_hi=3000, holes=0.0)
+    idx = a["idx"]
+    idx[0, 300:340] = idx[0, 5]
+    idx[1, 100:400:3] = idx[1, 100:200]
+    scale = 2.0 / math.sqrt(512)
+    out, lse = _run(a, cuda_device, scale)
+    _check(a, out, lse, scale)
+
+
 def test_sharp_softmax(cuda_device):
     # a large score factor: the chunk maxima differ by many units, exercising
     # the rescaling of the combine step

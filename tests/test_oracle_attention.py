@@ -2,8 +2,8 @@
 
 Checked against a library routine (torch's scaled_dot_product_attention in
 float64 when every cache row is selected), closed forms (identical rows, zero
-queries, a two-row case worked by hand, the sink's share, empty inputs) and
-invariants (slot order, skipped slots, moving a row between the cache and the
+queries, a two-row case worked by hand, a repeated slot, the sink's share, empty
+inputs) and invariants (slot order, skipped slots, moving a row between the cache and the
 window, per-batch caches, the scale folded into q, convexity).  Mutated copies
 of the attention rule are shown to fail the pins.
 """
@@ -200,6 +200,30 @@ def test_scale_folds_into_the_queries():
     assert np.allclose(a[0], b[0], rtol=1e-13, atol=1e-15) and np.allclose(a[1], b[1], rtol=1e-14)
 
 
+def test_repeated_slot_counts_once_per_slot():
+    # slots [0, 0, 1] with z = (1, 1, 0): row 0 carries weight 2e / (2e + 1)
+    q = bf16([[[2.0, 0.0]]])
+    kv = bf16([[1.0, 0.0], [0.0, 1.0]])
+    out, lse = sparse_attention(q, kv, np.array([[0, 0, 1]]), 0.5)
+    e2 = 2.0 * math.e
+    assert abs(out[0, 0, 0] - e2 / (e2 + 1.0)) < 1e-15
+    assert abs(out[0, 0, 1] - 1.0 / (e2 + 1.0)) < 1e-15
+    assert abs(lse[0, 0] - math.log(e2 + 1.0)) < 1e-14
+
+
+def test_repeated_slot_equals_the_row_also_in_the_window():
+    q, kv, win, idx, sink = _case(20, W=3)
+    rep = idx.copy()
+    rep[:, -1] = rep[:, 0]                       # the last slot repeats the first
+    w2 = win.copy()
+    for b in range(q.shape[0]):
+        w2[b, 0] = kv[idx[b, 0]]                 # the same row as the window's only row
+    a = sparse_attention(q, kv, rep, 0.3, win=win, win_len=np.zeros(2, np.int32), sink=sink)
+    c = sparse_attention(q, kv, idx[:, :-1], 0.3, win=w2,
+                         win_len=np.ones(2, np.int32), sink=sink)
+    assert np.allclose(a[0], c[0], atol=1e-13) and np.allclose(a[1], c[1], atol=1e-13)
+
+
 def test_output_is_inside_the_rows_hull():
     q, kv, win, idx, _ = _case(18, with_sink=False)
     out, _ = sparse_attention(q, kv, idx, 2.0, win=win)
@@ -217,6 +241,9 @@ def _pins_pass(fn):
     kv = bf16([[1.0, 0.0], [0.0, 1.0]])
     o, l = fn(q, kv, np.array([[1, 0]]), 0.5, None, None, None)
     if not (abs(o[0, 0, 0] - 0.7310585786300049) < 1e-12 and abs(l[0, 0] - 1.3132616875182228) < 1e-12):
+        return False
+    o, l = fn(q, kv, np.array([[0, 0, 1]]), 0.5, None, None, None)
+    if abs(o[0, 0, 0] - 2 * math.e / (2 * math.e + 1)) > 1e-12:
         return False
     o, l = fn(np.zeros((1, 1, 2), np.uint16), kv, np.array([[0, 1]]), 1.0, None, None, np.array([math.log(2)]))
     if not np.allclose(o[0, 0], _dec(kv).mean(0) / 2, atol=1e-12):
@@ -264,11 +291,23 @@ def _m_sqrt_scale(q, kv, idx, scale, win, wl, sink):
     return sparse_attention(q, kv, idx, math.sqrt(scale), win=win, win_len=wl, sink=sink)
 
 
+def _m_dedup_slots(q, kv, idx, scale, win, wl, sink):
+    # a row selected by several slots attended once
+    d = np.array(idx).copy()
+    for b in range(d.shape[0]):
+        seen = set()
+        for j in range(d.shape[1]):
+            if int(d[b, j]) in seen:
+                d[b, j] = -1
+            seen.add(int(d[b, j]))
+    return sparse_attention(q, kv, d, scale, win=win, win_len=wl, sink=sink)
+
+
 def test_pins_accept_the_oracle():
     assert _pins_pass(_correct)
 
 
 @pytest.mark.parametrize("mutant", [_m_sink_carries_value, _m_separate_softmax, _m_window_of_batch0,
-                                    _m_sqrt_scale])
+                                    _m_sqrt_scale, _m_dedup_slots])
 def test_pins_catch_planted_mistakes(mutant):
     assert not _pins_pass(mutant)
