@@ -1,5 +1,6 @@
-"""Host-side logic of bench.py (CPU only): algorithmic byte / FLOP counts, the
-clock-log summary, and the max-over-ranks reduction with two gloo ranks."""
+"""Host-side logic of bench.py (CPU only): algorithmic byte / FLOP counts (top-k,
+decode step, sparse attention), the clock-log summary, and the max-over-ranks
+reduction with two gloo ranks."""
 
 import os
 import socket
@@ -21,6 +22,24 @@ def test_decode_bytes_and_flops():
     b, f = bench.decode_bytes_flops(vl, 64, 128, 1024)
     assert f == 2 * 64 * 128 * int(vl.sum())
     assert b == 32768 * 256 + 3 * 64 * 128 * 2 + 3 * 64 * 4 + 3 * 4 + 3 * 1024 * 4
+
+
+def test_attention_bytes_and_flops_decode_workload():
+    # 8 rows x (1024 selected + 128 window) rows of 512 bf16 channels, read once;
+    # q read and out written (8 x 128 x 512 bf16 each), lse, slots, sink, win_len
+    idx = np.arange(8 * 1024, dtype=np.int32).reshape(8, 1024)
+    b, f = bench.attention_bytes_flops(idx, 32768, np.full(8, 128), 128, 512, 1024)
+    assert b == 9437184 + 2097152 + 4096 + 32768 + 512 + 32 == 11571744
+    assert f == 4 * 128 * 512 * 9216
+
+
+def test_attention_bytes_skip_invalid_slots():
+    # -1 padding and slots at or past T attend nothing and read no row
+    idx = np.array([[0, -1, 5, 9], [10, 3, -1, -1]], dtype=np.int32)
+    b, f = bench.attention_bytes_flops(idx, 9, np.array([2, 0]), 4, 64, 4)
+    rows = 2 + 1 + 2                      # T = 9: (0, 5) and (3) valid; 2 window rows
+    assert f == 4 * 4 * 64 * rows
+    assert b == rows * 64 * 2 + 2 * 2 * 4 * 64 * 2 + 2 * 4 * 4 + 2 * 4 * 4 + 4 * 4 + 2 * 4
 
 
 def test_clock_summary_flags_throttle_reasons():
