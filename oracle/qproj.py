@@ -50,8 +50,11 @@ def qproj(x_bits, wq_bits, ww_bits=None, heads=None, d=128):
 def round_bf16(v):
     """Round float64 values to the nearest bfloat16 (ties to even), as float64.
 
-    Exact: the value is first rounded to float32's grid only where that cannot
-    change the bfloat16 result, which is checked by comparing both neighbours.
+    The neighbours are the two multiples of the quantum around the value: the
+    quantum is 2^(e - 7) for a value in [2^e, 2^(e+1)) (8 significant bits), and
+    2^-133 below 2^-126, where bfloat16 (binary32's exponent range) is subnormal.
+    A result of magnitude 2^128 or more is past the largest finite bfloat16,
+    (2 - 2^-7) * 2^127, and becomes infinity; a zero result keeps the sign.
     """
     v = np.asarray(v, dtype=np.float64)
     out = np.empty_like(v)
@@ -63,6 +66,7 @@ def round_bf16(v):
         e = np.floor(np.log2(abs(a)))
         if abs(a) < 2.0 ** e:                     # log2 rounded up just below a power of two
             e -= 1
+        e = max(e, -126.0)                        # the subnormal range's fixed quantum
         ulp = 2.0 ** (e - 7)                      # bfloat16 keeps 8 significant bits
         lo = np.floor(a / ulp) * ulp
         hi = lo + ulp
@@ -72,4 +76,8 @@ def round_bf16(v):
             res[i] = hi
         else:                                     # a tie: the even significand
             res[i] = lo if int(round(lo / ulp)) % 2 == 0 else hi
+        if abs(res[i]) >= 2.0 ** 128:
+            res[i] = np.copysign(np.inf, a)
+        elif res[i] == 0:
+            res[i] = np.copysign(0.0, a)
     return out

@@ -91,6 +91,29 @@ def test_round_bf16_matches_the_generators_rounding():
         assert np.array_equal(got, ref)
 
 
+def test_round_bf16_subnormals_and_overflow():
+    g = np.random.default_rng(5)
+    # bfloat16 subnormals (below 2^-126, quantum 2^-133), values halfway between
+    # two of them, and the boundary to the normal range
+    sub = (g.standard_normal(5000) * 2.0 ** -131).astype(np.float32)
+    kk = g.integers(-127, 128, 500).astype(np.float64)
+    sub_ties = ((kk + 0.5) * 2.0 ** -133).astype(np.float32)
+    edge = np.array([2.0 ** -126, 2.0 ** -126 - 2.0 ** -134, 2.0 ** -134, -2.0 ** -134, 3 * 2.0 ** -134,
+                     2.0 ** -149], dtype=np.float32)
+    # the top: the largest finite bfloat16, the tie above it (rounds to even:
+    # infinity), and the largest float32
+    big = (2.0 - 2.0 ** -7) * 2.0 ** 127
+    top = np.array([big, -big, big + 2.0 ** 118, (2.0 - 2.0 ** -8) * 2.0 ** 127, 3.4028234663852886e38],
+                   dtype=np.float32)
+    for arr in (sub, sub_ties, edge, top):
+        ref = _dec(bf16(arr))
+        got = round_bf16(arr.astype(np.float64))
+        assert np.array_equal(got, ref)
+        assert np.array_equal(np.signbit(got), np.signbit(ref))
+    assert np.isinf(round_bf16(np.array([(2.0 - 2.0 ** -8) * 2.0 ** 127]))[0])
+    assert round_bf16(np.array([big]))[0] == big
+
+
 def _correct(x, wq, heads, d):
     return qproj(x, wq, heads=heads, d=d)[0]
 
