@@ -410,7 +410,7 @@ static bool encode_maps(const void* q, const void* kc, int B, int H, int S, int 
 // Keys viewed as (64 channels, S positions, 2 channel halves, nk caches),
 // caches kstride rows apart, in boxes of (64, 128, 2, 1): one copy is a whole
 // 128-position tile, its two 64-channel halves one after the other.
-static bool encode_kmap3(const void* kc, int S, int nk, long long kstride, CUtensorMap* tk) {
+static bool encode_kmap(const void* kc, int S, int nk, long long kstride, CUtensorMap* tk) {
   cuuint64_t dims[4] = {64, (cuuint64_t)S, 2, (cuuint64_t)nk};
   cuuint64_t str[3] = {256, 128, (cuuint64_t)(kstride > 0 ? kstride : S) * 256};
   cuuint32_t box[4] = {64, 128, 2, 1};
@@ -428,7 +428,7 @@ static int launch_score(const void* q, const void* kc, const float* w, int B, in
   if (!encode_maps(q, kc, B, H, S, HP, NT, &tq, &tk)) return DS_ERR_ARG;
   const bool per_row = kstride > 0;
   if (per_row && NT != 1) return DS_ERR_ARG;
-  if (!encode_kmap3(kc, S, per_row ? B : 1, kstride, &tk)) return DS_ERR_ARG;
+  if (!encode_kmap(kc, S, per_row ? B : 1, kstride, &tk)) return DS_ERR_ARG;
   const int ntiles = (S + 127) / 128;
   const int groups = (B + NT - 1) / NT;
   // spread one group's tiles over several CTAs only while there are fewer
