@@ -237,6 +237,24 @@ def ds_indexer_topk(q, kcache, w, k, valid_len=None, return_score=False,
     return out_idx, (out_score if return_score else None)
 
 
+def ds_indexer_topk_noalloc(q, kcache, w, k, valid_len=None, return_score=False,
+                            out_idx=None, out_score=None, stream=None):
+    """ds_indexer_topk through the allocation-free entry point (batch * S <= 262144)."""
+    import torch
+    dev, batch, heads, d, S = _indexer_args(q, kcache, w, valid_len)
+    if out_idx is None:
+        out_idx = torch.empty((batch, k), dtype=torch.int32, device=dev)
+    _require(out_idx, torch.int32, "out_idx", dev)
+    if return_score and out_score is None:
+        out_score = torch.empty((batch, k), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        rc = ds_indexer_topk_noalloc_raw(_ptr(q), _ptr(kcache), _ptr(w), batch, heads, d, S,
+                                         _ptr(valid_len), k, _ptr(out_idx),
+                                         _ptr(out_score) if return_score else None, _stream_ptr(stream))
+    _check(rc, "ds_indexer_topk_noalloc")
+    return out_idx, (out_score if return_score else None)
+
+
 def ds_sparse_attention(q, kv, idx, scale=None, win=None, win_len=None, sink=None, return_lse=False,
                         out=None, lse=None, stream=None):
     """Multi-query attention of every query head over the selected cache rows

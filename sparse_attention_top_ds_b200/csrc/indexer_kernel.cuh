@@ -27,27 +27,39 @@
 //    64-channel halves one after the other as the MMA reads them.  There is one
 //    cache for every row, or one per row (then a group is one row and reads
 //    cache t).
+//
+// With the selection (SEL = true; NKI pull request, "The top-k on the GPSIMD
+// engine": the index scores feed the top-k as they are produced):
+//  * The epilogue also counts every valid score of its rows in a shared-memory
+//    histogram of the top 12 bits of its order-preserving key (16-bit counters,
+//    two per word), and at the end adds the CTA's counts into the rows' global
+//    histograms; only valid positions are stored.
+//  * topk_hist_select_kernel (select_phase.cuh) then starts from the exact
+//    threshold bin those histograms give: one pass over each row, no sampling
+//    and no histogram pass of its own.
 #pragma once
 
 #include <cuda.h>
 
 #include "ptx.cuh"
 #include "tcgen05.cuh"
+#include "select_phase.cuh"
 
 namespace dstopk {
 
 struct ScoreParams {
   const float* w;           // [B, H]
   const int32_t* valid_len; // [B] or null
-  float* out;               // [B, S]
+  float* out;               // [B, S]: every score (SEL: valid positions only, read back by the selection)
   int* status;
   int B, H, S;
   int tiles_per_cta;        // 128-position tiles per CTA
   int ctas_per_group;       // CTAs sharing one group of NT rows
   int key_per_row;          // 1: row t reads key cache t (then NT == 1); 0: one cache for every row
+  uint32_t* ghist;          // SEL: [B, 4096] key histograms, zero before the launch
 };
 
-template <int NT, int HP, int STAGES>
+template <int NT, int HP, int STAGES, bool SEL = false>
 struct ScoreCfg {
   static constexpr int kN = NT * HP;                 // accumulator columns per tile
   static constexpr int kNmma = kN < 256 ? kN : 256;  // N of one MMA instruction
@@ -65,7 +77,9 @@ struct ScoreCfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + 2 * kQHalf;
   static constexpr int kOffW = kOffK + STAGES * kStage;
-  static constexpr int kOffBar = kOffW + NT * HP * 4;
+  static constexpr int kOffHist = kOffW + NT * HP * 4;          // SEL: u16 key histograms, 2 per word
+  static constexpr int kHistBytes = SEL ? NT * (kSelBins / 2) * 4 : 0;
+  static constexpr int kOffBar = kOffHist + kHistBytes;
   // barriers: qfull, kfull[STAGES], kempty[STAGES], afull[2], aempty[2], tmem slot
   static constexpr int kBarQ = 0;
   static constexpr int kBarKFull = 1;
@@ -77,13 +91,22 @@ struct ScoreCfg {
   static constexpr int kSmemBytes = kOffTmemSlot + 16 + 1024;  // + alignment slack
   static_assert(kN % 16 == 0 && kN <= 256 && kN % kNmma == 0, "bad tile");
   static_assert(HP % 16 == 0 && HP <= 64, "bad head padding");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+  // SEL: 16-bit histogram counters hold the positions one CTA scores per row
+  static constexpr int kMaxTilesPerCta = 65535 / 128;
 };
 
-template <int NT, int HP, int STAGES>
-__global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
+// valid positions of row t, clamped to [0, S]
+__device__ __forceinline__ int row_valid_len(const ScoreParams& p, int t) {
+  int v = p.valid_len ? p.valid_len[t] : p.S;
+  return v < 0 ? 0 : (v > p.S ? p.S : v);
+}
+
+template <int NT, int HP, int STAGES, bool SEL = false>
+__global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES, SEL>::kThreads, 1)
     indexer_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const ScoreParams p) {
-  using C = ScoreCfg<NT, HP, STAGES>;
+  using C = ScoreCfg<NT, HP, STAGES, SEL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -145,6 +168,10 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
   for (int i = threadIdx.x; i < NT * HP; i += C::kThreads) {
     const int t = i / HP, h = i % HP;
     w_s[i] = (t0 + t < p.B && h < p.H) ? p.w[(size_t)(t0 + t) * p.H + h] : 0.0f;
+  }
+  uint32_t* hist16 = reinterpret_cast<uint32_t*>(smem + C::kOffHist);  // SEL: [NT][2048] words
+  if constexpr (SEL) {
+    for (int i = threadIdx.x; i < NT * (kSelBins / 2); i += C::kThreads) hist16[i] = 0u;
   }
   tc_fence_before();
   __syncthreads();
@@ -233,14 +260,24 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
 #pragma unroll
         for (int x = 0; x < HP; ++x) acc = fmaf(w_s[tl * HP + x], fmaxf(__uint_as_float(r[x]), 0.0f), acc);
         const int t = t0 + tl;
-        if (t < p.B && s < p.S) p.out[(size_t)t * p.S + s] = (s < vl[j]) ? acc : -INFINITY;
+        if constexpr (SEL) {
+          // valid positions: counted, and stored for the selection
+          if (t < p.B && s < vl[j]) {
+            const uint32_t bin = F32Keys::key(__float_as_uint(acc)) >> kSelShift;
+            atomicAdd(hist16 + tl * (kSelBins / 2) + (bin >> 1), 1u << ((bin & 1u) << 4));
+            p.out[(size_t)t * p.S + s] = acc;
+          }
+        } else {
+          if (t < p.B && s < p.S) p.out[(size_t)t * p.S + s] = (s < vl[j]) ? acc : -INFINITY;
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::kBarAEmpty + slot));
     }
-    // tiles past the group's valid lengths: no products, -inf
-    for (int tile = act_hi > tile_lo ? act_hi : tile_lo; tile < tile_hi; ++tile) {
+    // tiles past the group's valid lengths: no products, -inf (the selection
+    // never reads them)
+    for (int tile = act_hi > tile_lo ? act_hi : tile_lo; !SEL && tile < tile_hi; ++tile) {
       const int s = tile * 128 + row;
 #pragma unroll
       for (int j = 0; j < TPH; ++j) {
@@ -255,8 +292,20 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
-  // the next kernel (the top-k over these rows) may launch only now: launched
-  // earlier its CTAs would crowd onto the few SMs this grid leaves free
+  if constexpr (SEL) {
+    // every score is counted: add this CTA's counts into the rows' global
+    // histograms (the selection kernel reads them once this grid has finished)
+    for (int tl = 0; tl < NT && t0 + tl < p.B; ++tl) {
+      uint32_t* gh = p.ghist + (size_t)(t0 + tl) * kSelBins;
+      for (int i = threadIdx.x; i < kSelBins / 2; i += C::kThreads) {
+        const uint32_t v = hist16[tl * (kSelBins / 2) + i];
+        if (v & 0xFFFFu) atomicAdd(gh + 2 * i, v & 0xFFFFu);
+        if (v >> 16) atomicAdd(gh + 2 * i + 1, v >> 16);
+      }
+    }
+  }
+  // the next kernel (the selection over these rows) may launch only now:
+  // launched earlier its CTAs would crowd onto the few SMs this grid leaves free
   pdl_launch_dependents();
 }
 

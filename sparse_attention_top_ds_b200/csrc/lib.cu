@@ -16,8 +16,6 @@
 #include "topk_kernel.cuh"
 #include "topk_stash_kernel.cuh"
 #include "indexer_kernel.cuh"
-#include "decode_kernel.cuh"
-#include "rowcluster_kernel.cuh"
 #include "attention_kernel.cuh"
 #include "qproj_kernel.cuh"
 #include "compress_kernel.cuh"
@@ -34,14 +32,10 @@ struct DeviceState {
   bool supported = false;
   int num_sms = 0;
   int* status = nullptr;     // device address of g_status on this device
-  void* scratch = nullptr;   // grow-only scratch for ds_indexer_topk
+  void* scratch = nullptr;   // grow-only scratch: [B, S] score rows of the indexer paths
   size_t scratch_bytes = 0;
-  uint32_t* dec_ctl = nullptr;   // fused decode: control table (two copies, zeroed once)
-  uint32_t* dec_cand = nullptr;  // fused decode: candidate lists, grow-only
-  size_t dec_cand_bytes = 0;
-  int dec_max_blocks = 0;        // co-resident CTAs of the fused decode kernel
-  int rc_cluster = 0;            // row-per-cluster indexer + top-k: CTAs per row (0: unavailable)
-  int rc_active = 0;             // clusters of that size the device runs at once
+  void* sel_state = nullptr;  // indexer + top-k: key histograms of the rows (zero between calls)
+  size_t sel_state_bytes = 0;
   void* attn_scratch = nullptr;  // sparse attention: per-chunk partial results, grow-only
   size_t attn_scratch_bytes = 0;
 };
@@ -58,7 +52,6 @@ static cudaError_t set_stash_smem(int bytes) {
   return e;
 }
 static bool topk_cluster16_ok();
-static int rowcluster_active(int C);
 static int g_max_cluster = 8;  // largest cluster the top-k launch may use
 
 // Launch attribute: the kernel may start while the previous kernel on the
@@ -101,10 +94,6 @@ static int device_state(DeviceState** out) {
       if (e == cudaSuccess) e = indexer_setup();
       if (e != cudaSuccess) return DS_ERR_CUDA;
       g_max_cluster = topk_cluster16_ok() ? 16 : 8;
-      const int a16 = rowcluster_active(16);
-      const int a8 = a16 > 0 ? 0 : rowcluster_active(8);
-      s.rc_cluster = a16 > 0 ? 16 : (a8 > 0 ? 8 : 0);
-      s.rc_active = a16 > 0 ? a16 : a8;
     }
     s.ready = true;
   }
@@ -162,6 +151,7 @@ static bool topk_cluster16_ok() {
   cudaFuncSetAttribute(topk_cluster_kernel<F32Keys, 512>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   cudaFuncSetAttribute(topk_cluster_kernel<BF16Keys, 256>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   cudaFuncSetAttribute(topk_cluster_kernel<BF16Keys, 512>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaFuncSetAttribute(topk_hist_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(16, 1, 1);
@@ -316,10 +306,10 @@ static const PvCfg* pv_pick(int NS) {
   return nullptr;
 }
 
-template <int NT, int HP, int ST>
+template <int NT, int HP, int ST, bool SEL = false>
 static cudaError_t set_score_smem() {
-  return cudaFuncSetAttribute(indexer_score_kernel<NT, HP, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              ScoreCfg<NT, HP, ST>::kSmemBytes);
+  return cudaFuncSetAttribute(indexer_score_kernel<NT, HP, ST, SEL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              ScoreCfg<NT, HP, ST, SEL>::kSmemBytes);
 }
 
 // Called once per device from device_state (under its lock).
@@ -338,12 +328,15 @@ static cudaError_t indexer_setup() {
   if (e == cudaSuccess) e = set_score_smem<8, 16, 4>();
   if (e == cudaSuccess) e = set_score_smem<1, 32, 4>();
   if (e == cudaSuccess) e = set_score_smem<1, 16, 4>();
+  if (e == cudaSuccess) e = set_score_smem<1, 64, 4, true>();
+  if (e == cudaSuccess) e = set_score_smem<2, 64, 4, true>();
+  if (e == cudaSuccess) e = set_score_smem<4, 64, 4, true>();
+  if (e == cudaSuccess) e = set_score_smem<1, 32, 4, true>();
+  if (e == cudaSuccess) e = set_score_smem<1, 16, 4, true>();
+  if (e == cudaSuccess) e = set_score_smem<4, 32, 4, true>();
+  if (e == cudaSuccess) e = set_score_smem<4, 16, 4, true>();
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(indexer_topk_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DecodeSmem::kBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(indexer_topk_rowcluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             RcSmem::kBytes);
+    e = cudaFuncSetAttribute(topk_hist_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HsSmem::kBytes);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(sparse_attn_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              AttnSmem::bytes(kAttnMaxD));
@@ -355,34 +348,6 @@ static cudaError_t indexer_setup() {
   for (int i = 0; e == cudaSuccess && i < kPvCfgs; ++i)
     e = cudaFuncSetAttribute(kPvCfg[i].fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   return e;
-}
-
-// Clusters the row-per-cluster kernel can run at once with C CTAs each (0 if none).
-static int rowcluster_active(int C) {
-  if (C == 16 &&
-      cudaFuncSetAttribute(indexer_topk_rowcluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-          cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3((unsigned)C, 1, 1);
-  cfg.blockDim = dim3(kRcThreads, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)RcSmem::kBytes;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, indexer_topk_rowcluster_kernel, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  return n;
 }
 
 // bf16 tensor maps with 128-byte swizzle: queries [B][H][128] in boxes of
@@ -489,135 +454,6 @@ static int score_enqueue(const void* q, const void* kc, const float* w, int B, i
   return launch_score<8, 16, 4>(q, kc, w, B, H, S, vl, out, 0, st, s);
 }
 
-// ---- fused decode (score + top-k in one cooperative launch)
-
-// The single-launch grid-wide variant is opt-in (DS_INDEXER_FUSED=1): on this
-// GPU its chain of grid-wide round trips costs more than the two-kernel path.
-static bool decode_fits(int B, int H, int S, const DeviceState* s) {
-  if (getenv("DS_INDEXER_UNFUSED")) return false;  // testing / comparison only
-  if (!getenv("DS_INDEXER_FUSED")) return false;
-  if (B > kDecRows || H <= 32 || H > kDecHeads) return false;
-  const int ntiles = (S + 127) / 128;
-  return ntiles <= s->num_sms * kDecMaxTiles;
-}
-
-static int decode_enqueue(const void* q, const void* kc, const float* w, int B, int H, int S,
-                          const int32_t* vl, int k, int32_t* out_idx, float* out_score, cudaStream_t st,
-                          DeviceState* s) {
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!s->dec_ctl) {
-      void* p = nullptr;
-      if (cudaMalloc(&p, DecodeCtl::kTotal * sizeof(uint32_t)) != cudaSuccess) {
-        cudaGetLastError();
-        return DS_ERR_NOMEM;
-      }
-      if (cudaMemset(p, 0, DecodeCtl::kTotal * sizeof(uint32_t)) != cudaSuccess) return DS_ERR_CUDA;
-      s->dec_ctl = static_cast<uint32_t*>(p);
-      int per_sm = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, indexer_topk_decode_kernel, kDecThreads,
-                                                        DecodeSmem::kBytes) != cudaSuccess)
-        return DS_ERR_CUDA;
-      s->dec_max_blocks = per_sm * s->num_sms;
-    }
-    const size_t need = (size_t)B * (size_t)S * 2 * sizeof(uint32_t);
-    if (s->dec_cand_bytes < need) {
-      if (s->dec_cand) cudaFree(s->dec_cand);
-      s->dec_cand = nullptr;
-      s->dec_cand_bytes = 0;
-      void* p = nullptr;
-      if (cudaMalloc(&p, need) != cudaSuccess) {
-        cudaGetLastError();
-        return DS_ERR_NOMEM;
-      }
-      s->dec_cand = static_cast<uint32_t*>(p);
-      s->dec_cand_bytes = need;
-    }
-  }
-  const int ntiles = (S + 127) / 128;
-  int G = min(ntiles, min(s->num_sms, s->dec_max_blocks));
-  if (G < 1) return DS_ERR_CUDA;
-  const int tpc = (ntiles + G - 1) / G;
-  if (tpc > kDecMaxTiles) return DS_ERR_ARG;
-  G = (ntiles + tpc - 1) / tpc;
-  CUtensorMap tq, tk;
-  if (!encode_maps(q, kc, B, H, S, kDecHeads, 4, &tq, &tk)) return DS_ERR_ARG;
-  DecodeParams p;
-  p.w = w;
-  p.valid_len = vl;
-  p.out_idx = out_idx;
-  p.out_score = out_score;
-  p.status = s->status;
-  p.B = B;
-  p.H = H;
-  p.S = S;
-  p.k = k;
-  p.tiles_per_cta = tpc;
-  p.ctl = s->dec_ctl;
-  p.cand = s->dec_cand;
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3((unsigned)G, 1, 1);
-  cfg.blockDim = dim3(kDecThreads, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)DecodeSmem::kBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, indexer_topk_decode_kernel, tq, tk, p);
-  return e == cudaSuccess ? DS_OK : DS_ERR_CUDA;
-}
-
-// ---- row-per-cluster indexer + top-k (one launch, nothing written but the result)
-
-// Opt-in (DS_INDEXER_ROWCLUSTER=1): with one 16-CTA cluster per row each SM
-// streams 1/16 of the row's keys at the rate one SM reaches alone, and the
-// leader's pass over the row is latency bound, so on this GPU the two-kernel
-// path is faster at every batch size measured (1 to 64 rows).
-static bool rowcluster_fits(int B, int H, int S, const DeviceState* s) {
-  if (s->rc_cluster == 0 || S > kRcMaxS || H > kRcHeads || B <= 0) return false;
-  const char* f = getenv("DS_INDEXER_ROWCLUSTER");
-  return f && atoi(f) == 1;
-}
-
-static int rowcluster_enqueue(const void* q, const void* kc, const float* w, int B, int H, int S,
-                              const int32_t* vl, int k, int32_t* out_idx, float* out_score, cudaStream_t st,
-                              DeviceState* s) {
-  const int C = s->rc_cluster;
-  const int ppc = ((S + C - 1) / C + 127) / 128 * 128;
-  if (ppc > kRcMaxPPC || (long)ppc * C < S) return DS_ERR_ARG;
-  CUtensorMap tq, tk;
-  if (!encode_maps(q, kc, B, H, S, kRcHeads, 1, &tq, &tk)) return DS_ERR_ARG;
-  RowClusterParams p;
-  p.w = w;
-  p.valid_len = vl;
-  p.out_idx = out_idx;
-  p.out_score = out_score;
-  p.status = s->status;
-  p.B = B;
-  p.H = H;
-  p.S = S;
-  p.k = k;
-  p.ppc = ppc;
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3((unsigned)(B * C), 1, 1);
-  cfg.blockDim = dim3(kRcThreads, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)RcSmem::kBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)C;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, indexer_topk_rowcluster_kernel, tq, tk, p);
-  return e == cudaSuccess ? DS_OK : DS_ERR_CUDA;
-}
-
 static int indexer_check(const void* q, const void* kc, const float* w, int B, int H, int d, int S) {
   if (!q || !kc || !w || B <= 0 || H <= 0 || H > DS_INDEXER_MAX_HEADS || d != DS_INDEXER_DIM || S <= 0)
     return DS_ERR_ARG;
@@ -642,6 +478,167 @@ static void* get_scratch(DeviceState* s, size_t bytes) {
   s->scratch = p;
   s->scratch_bytes = bytes;
   return p;
+}
+
+// ---- indexer + top-k (the path of ds_indexer_topk and ds_indexer_topk_ex)
+//
+// Rows split over several scorer CTAs (few rows, as in decode): the scorer
+// also counts every valid score in an exact histogram of its key's top 12 bits
+// (per row, added into global memory), and topk_hist_select_kernel starts from
+// the threshold bin those counts give: no sampling and no histogram pass of
+// its own.  Whole rows per scorer CTA (many rows, as in prefill): the scores
+// go to the [B, S] buffer and ds_topk's kernel selects them; on this GPU that
+// measured faster than selecting inside the scorer's CTAs (whose selection
+// tail leaves the tensor pipe idle) or beside them.
+
+// Grow-only buffer that is all zero whenever no call is in flight: zeroed when
+// (re)allocated, and every launch that uses it leaves it zero again.
+static void* get_zeroed_state(DeviceState* s, size_t bytes) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (s->sel_state_bytes >= bytes) return s->sel_state;
+  if (s->sel_state) cudaFree(s->sel_state);
+  s->sel_state = nullptr;
+  s->sel_state_bytes = 0;
+  void* p = nullptr;
+  if (cudaMalloc(&p, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (cudaMemset(p, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaFree(p);
+    return nullptr;
+  }
+  s->sel_state = p;
+  s->sel_state_bytes = bytes;
+  return p;
+}
+
+// Scorer CTAs per group of NT rows for the scores-with-histograms launch (the
+// same spread as score_enqueue's, capped by the 16-bit counters).
+template <int NT, int HP, int ST>
+static int hist_groups_split(int B, int S, const DeviceState* s, int* tpc_out) {
+  using Cfg = ScoreCfg<NT, HP, ST, true>;
+  const int ntiles = (S + 127) / 128;
+  const int groups = (B + NT - 1) / NT;
+  long tpc = ((long)groups * ntiles + s->num_sms - 1) / s->num_sms;
+  tpc = std::max(1L, std::min(tpc, (long)std::min(ntiles, Cfg::kMaxTilesPerCta)));
+  *tpc_out = (int)tpc;
+  return (int)((ntiles + tpc - 1) / tpc);
+}
+
+// One scorer launch: scores of the valid positions to out [B, S], key counts
+// added into ghist [B, 4096].
+template <int NT, int HP, int ST>
+static int launch_score_hist(const void* q, const void* kc, const float* w, int B, int H, int S, const int32_t* vl,
+                             long long kstride, float* out, uint32_t* ghist, cudaStream_t st, DeviceState* s) {
+  using Cfg = ScoreCfg<NT, HP, ST, true>;
+  CUtensorMap tq, tk;
+  if (!encode_maps(q, kc, B, H, S, HP, NT, &tq, &tk)) return DS_ERR_ARG;
+  const bool per_row = kstride > 0;
+  if (per_row && NT != 1) return DS_ERR_ARG;
+  if (!encode_kmap(kc, S, per_row ? B : 1, kstride, &tk)) return DS_ERR_ARG;
+  int tpc = 0;
+  const int cpg = hist_groups_split<NT, HP, ST>(B, S, s, &tpc);
+  ScoreParams p;
+  memset(&p, 0, sizeof(p));
+  p.w = w;
+  p.valid_len = vl;
+  p.out = out;
+  p.status = s->status;
+  p.B = B;
+  p.H = H;
+  p.S = S;
+  p.tiles_per_cta = tpc;
+  p.ctas_per_group = cpg;
+  p.key_per_row = per_row ? 1 : 0;
+  p.ghist = ghist;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)(((B + NT - 1) / NT) * cpg), 1, 1);
+  cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)Cfg::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  set_pdl(attr[0]);
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_on() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, indexer_score_kernel<NT, HP, ST, true>, tq, tk, p) == cudaSuccess ? DS_OK
+                                                                                                    : DS_ERR_CUDA;
+}
+
+// One selection launch over B rows: a cluster of C CTAs per row, as many as
+// keep every slice at 1024 scores or more and the rows' CTAs within the SM count.
+static int launch_hist_select(const float* scores, uint32_t* ghist, const int32_t* vl, int32_t* out_idx,
+                              float* out_score, int B, int S, int k, int sorted, cudaStream_t st, DeviceState* s) {
+  int C = 1;
+  while (2 * C <= g_max_cluster && (long)B * 2 * C <= s->num_sms && S / (2 * C) >= 1024) C *= 2;
+  HsParams h;
+  memset(&h, 0, sizeof(h));
+  h.scores = scores;
+  h.ghist = ghist;
+  h.valid_len = vl;
+  h.out_idx = out_idx;
+  h.out_score = out_score;
+  h.B = B;
+  h.S = S;
+  h.k = k;
+  h.slice = ((S + C - 1) / C + 3) / 4 * 4;
+  h.sorted = sorted;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)(B * C), 1, 1);
+  cfg.blockDim = dim3(kHsThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)HsSmem::kBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  set_pdl(attr[1]);
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_on() ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, topk_hist_select_kernel, h) == cudaSuccess ? DS_OK : DS_ERR_CUDA;
+}
+
+template <int NT, int HP, int ST>
+static int indexer_topk_rows(const void* q, const void* kc, const float* w, int B, int H, int S, const int32_t* vl,
+                             int k, int sorted, int32_t* out_idx, float* out_score, long long kstride,
+                             cudaStream_t st, DeviceState* s) {
+  float* sc = static_cast<float*>(get_scratch(s, (size_t)B * (size_t)S * sizeof(float)));
+  if (!sc) return DS_ERR_NOMEM;
+  int tpc = 0;
+  if (hist_groups_split<NT, HP, ST>(B, S, s, &tpc) > 1) {
+    uint32_t* gh = static_cast<uint32_t*>(get_zeroed_state(s, (size_t)B * kSelBins * sizeof(uint32_t)));
+    if (!gh) return DS_ERR_NOMEM;
+    const int rc = launch_score_hist<NT, HP, ST>(q, kc, w, B, H, S, vl, kstride, sc, gh, st, s);
+    if (rc != DS_OK) return rc;
+    return launch_hist_select(sc, gh, vl, out_idx, out_score, B, S, k, sorted, st, s);
+  }
+  const int rc = score_enqueue(q, kc, w, B, H, S, vl, sc, st, s, kstride);
+  if (rc != DS_OK) return rc;
+  return topk_enqueue(sc, B, S, k, DS_F32, vl, out_idx, out_score, out_score != nullptr, sorted, st, s);
+}
+
+// Rows per CTA group: as for the scores alone (two rows for 2 and 5..8 rows,
+// one for one row, four otherwise); one row with a key cache per row; four
+// rows with 32 or fewer heads (N = 128 or 64).
+static int fused_enqueue(const void* q, const void* kc, const float* w, int B, int H, int S, const int32_t* vl,
+                         int k, int sorted, int32_t* out_idx, float* out_score, long long kstride, cudaStream_t st,
+                         DeviceState* s) {
+  if (kstride > 0) {
+    if (H > 32) return indexer_topk_rows<1, 64, 4>(q, kc, w, B, H, S, vl, k, sorted, out_idx, out_score, kstride, st, s);
+    if (H > 16) return indexer_topk_rows<1, 32, 4>(q, kc, w, B, H, S, vl, k, sorted, out_idx, out_score, kstride, st, s);
+    return indexer_topk_rows<1, 16, 4>(q, kc, w, B, H, S, vl, k, sorted, out_idx, out_score, kstride, st, s);
+  }
+  if (H > 32) {
+    if (B == 1) return indexer_topk_rows<1, 64, 4>(q, kc, w, B, H, S, vl, k, sorted, out_idx, out_score, 0, st, s);
+    if (B == 2 || (B >= 5 && B <= 8))
+      return indexer_topk_rows<2, 64, 4>(q, kc, w, B, H, S, vl, k, sorted, out_idx, out_score, 0, st, s);
+    return indexer_topk_rows<4, 64, 4>(q, kc, w, B, H, S, vl, k, sorted, out_idx, out_score, 0, st, s);
+  }
+  if (H > 16) return indexer_topk_rows<4, 32, 4>(q, kc, w, B, H, S, vl, k, sorted, out_idx, out_score, 0, st, s);
+  return indexer_topk_rows<4, 16, 4>(q, kc, w, B, H, S, vl, k, sorted, out_idx, out_score, 0, st, s);
 }
 
 // ---- sparse attention over the selected rows
@@ -878,20 +875,19 @@ extern "C" void ds_release(void) {
   int cur = -1;
   if (cudaGetDevice(&cur) != cudaSuccess) cur = -1;
   for (int d = 0; d < kMaxDevices; ++d) {
-    if (g_dev[d].scratch || g_dev[d].dec_ctl || g_dev[d].dec_cand || g_dev[d].attn_scratch) {
+    DeviceState& st = g_dev[d];
+    if (st.scratch || st.sel_state || st.attn_scratch) {
       if (cudaSetDevice(d) == cudaSuccess) {
-        if (g_dev[d].scratch) cudaFree(g_dev[d].scratch);
-        if (g_dev[d].dec_ctl) cudaFree(g_dev[d].dec_ctl);
-        if (g_dev[d].dec_cand) cudaFree(g_dev[d].dec_cand);
-        if (g_dev[d].attn_scratch) cudaFree(g_dev[d].attn_scratch);
+        if (st.scratch) cudaFree(st.scratch);
+        if (st.sel_state) cudaFree(st.sel_state);
+        if (st.attn_scratch) cudaFree(st.attn_scratch);
       }
-      g_dev[d].attn_scratch = nullptr;
-      g_dev[d].attn_scratch_bytes = 0;
-      g_dev[d].scratch = nullptr;
-      g_dev[d].scratch_bytes = 0;
-      g_dev[d].dec_ctl = nullptr;
-      g_dev[d].dec_cand = nullptr;
-      g_dev[d].dec_cand_bytes = 0;
+      st.attn_scratch = nullptr;
+      st.attn_scratch_bytes = 0;
+      st.scratch = nullptr;
+      st.scratch_bytes = 0;
+      st.sel_state = nullptr;
+      st.sel_state_bytes = 0;
     }
   }
   if (cur >= 0) cudaSetDevice(cur);
@@ -917,18 +913,8 @@ extern "C" int ds_indexer_topk(const void* q, const void* kcache, const float* w
   DeviceState* s = nullptr;
   rc = device_state(&s);
   if (rc != DS_OK) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (!getenv("DS_INDEXER_UNFUSED")) {
-    if (decode_fits(batch, heads, S, s))
-      return decode_enqueue(q, kcache, w, batch, heads, S, valid_len, k, out_idx, out_score, st, s);
-    if (rowcluster_fits(batch, heads, S, s))
-      return rowcluster_enqueue(q, kcache, w, batch, heads, S, valid_len, k, out_idx, out_score, st, s);
-  }
-  float* scores = static_cast<float*>(get_scratch(s, (size_t)batch * (size_t)S * sizeof(float)));
-  if (!scores) return DS_ERR_NOMEM;
-  rc = score_enqueue(q, kcache, w, batch, heads, S, valid_len, scores, st, s);
-  if (rc != DS_OK) return rc;
-  return topk_enqueue(scores, batch, S, k, DS_F32, valid_len, out_idx, out_score, out_score != nullptr, 0, st, s);
+  return fused_enqueue(q, kcache, w, batch, heads, S, valid_len, k, 0, out_idx, out_score, 0,
+                       static_cast<cudaStream_t>(stream), s);
 }
 
 // ------------------------------------------------------------------ allocation-free indexer + top-k
@@ -1057,13 +1043,8 @@ extern "C" int ds_indexer_topk_ex(const void* q, const void* kcache, int64_t kca
   DeviceState* s = nullptr;
   rc = device_state(&s);
   if (rc != DS_OK) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* scores = static_cast<float*>(get_scratch(s, (size_t)batch * (size_t)S * sizeof(float)));
-  if (!scores) return DS_ERR_NOMEM;
-  rc = score_enqueue(q, kcache, w, batch, heads, S, valid_len, scores, st, s, (long long)kcache_batch_stride);
-  if (rc != DS_OK) return rc;
-  return topk_enqueue(scores, batch, S, k, DS_F32, valid_len, out_idx, out_score, out_score != nullptr, sorted_index,
-                      st, s);
+  return fused_enqueue(q, kcache, w, batch, heads, S, valid_len, k, sorted_index, out_idx, out_score,
+                       (long long)kcache_batch_stride, static_cast<cudaStream_t>(stream), s);
 }
 
 extern "C" int ds_compress_fold(const void* rows, int batch, int D, int64_t rows_batch_stride, const void* gate,

@@ -9,7 +9,9 @@
 namespace dstopk {
 
 // Status codes written to the per-device status word (match include/ds_topk.h).
-constexpr int kErrTimeout = -3;
+constexpr int kErrCuda = -2;     // DS_ERR_CUDA: a launch found its set-up inconsistent
+constexpr int kErrTimeout = -3;  // DS_ERR_TIMEOUT
+constexpr int kErrInternal = kErrCuda;
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s

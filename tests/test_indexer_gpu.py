@@ -167,100 +167,44 @@ def test_indexer_argument_errors(cuda_device):
         ds.ds_indexer_topk(q, kc, w, 10)         # heads > 64
 
 
-# ---------------------------------------------------------------- fused decode path
+# ---------------------------------------------------------------- the fused path: whole rows and split rows
+#
+# ds_indexer_topk scores and selects in one launch.  A CTA group that owns its
+# rows whole (many rows, as in prefill) selects them itself; rows split over
+# several CTAs (few rows, as in decode) are selected by the group's last CTA from
+# the histograms every CTA added up.  ds_indexer_topk_noalloc runs the same
+# scorer arithmetic as two launches (scores to a buffer, then ds_topk), so both
+# must select the same positions and return the same scores.
 
-@pytest.fixture
-def grid_fused(monkeypatch):
-    # the single-launch, grid-barrier decode kernel (opt-in)
-    monkeypatch.setenv("DS_INDEXER_FUSED", "1")
+
+def _same_selection(a_idx, a_sc, b_idx, b_sc):
+    for t in range(a_idx.shape[0]):
+        assert np.array_equal(np.sort(a_idx[t]), np.sort(b_idx[t])), f"row {t}"
+        oa, ob = np.argsort(a_idx[t]), np.argsort(b_idx[t])
+        assert np.array_equal(a_sc[t][oa], b_sc[t][ob]), f"row {t}: scores"
 
 
-def test_fused_decode_matches_unfused_path(cuda_device, grid_fused, monkeypatch):
-    # B <= 8 rows and 33..64 heads take the fused single-launch kernel; the
-    # unfused path (scores to scratch, then ds_topk) computes the same float32
-    # scores in the same order, so both select the same positions exactly.
-    q, kc, w, vl = inputs.decode(seed=31)
+@pytest.mark.parametrize("B,S,k", [(8, 32768, 1024), (2, 20000, 2048), (1, 5000, 64), (5, 9000, 700)])
+def test_fused_matches_two_launch_path(cuda_device, B, S, k):
+    q, kc, w, vl = inputs.decode(seed=31 + B, batch=B, S=S, vl_lo=min(4096, S // 2), vl_hi=S)
     qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
-    fused, fs = ds.ds_indexer_topk(qd, kd, wd, 1024, valid_len=vd, return_score=True)
+    fused, fs = ds.ds_indexer_topk(qd, kd, wd, k, valid_len=vd, return_score=True)
     torch.cuda.synchronize()
-    monkeypatch.setenv("DS_INDEXER_UNFUSED", "1")
-    ref, rs = ds.ds_indexer_topk(qd, kd, wd, 1024, valid_len=vd, return_score=True)
+    two, ts = ds.ds_indexer_topk_noalloc(qd, kd, wd, k, valid_len=vd, return_score=True)
     torch.cuda.synchronize()
     assert ds.ds_get_device_status() == ds.DS_OK
-    f, r = fused.cpu().numpy(), ref.cpu().numpy()
-    for t in range(q.shape[0]):
-        assert np.array_equal(np.sort(f[t]), np.sort(r[t])), f"row {t}"
-        of, orr = np.argsort(f[t]), np.argsort(r[t])
-        assert np.array_equal(fs.cpu().numpy()[t][of], rs.cpu().numpy()[t][orr])
+    _same_selection(fused.cpu().numpy(), fs.cpu().numpy(), two.cpu().numpy(), ts.cpu().numpy())
 
 
-@pytest.mark.parametrize("B,S,k", [(1, 40000, 2048), (5, 7000, 512), (8, 128, 64), (2, 75000, 100)])
-def test_fused_decode_shapes(cuda_device, grid_fused, B, S, k):
-    q, kc, w = inputs.indexer_factors(seed=B * 3 + S, batch=B, n=S, heads=64)
-    g = np.random.default_rng(S)
-    vl = g.integers(0, S + 1, size=B).astype(np.int32)
-    vl[0] = S
-    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
-    idx, score = ds.ds_indexer_topk(qd, kd, wd, k, valid_len=vd, return_score=True)
-    torch.cuda.synchronize()
-    assert ds.ds_get_device_status() == ds.DS_OK
-    check_selection(q, kc, w, vl, k, idx.cpu().numpy(), score.cpu().numpy())
-
-
-def test_fused_decode_graph_replay_with_odd_call_count(cuda_device, grid_fused):
-    # the fused kernel alternates between two copies of its control table on
-    # its own; replaying a graph of 3 calls several times must keep results right
-    q, kc, w, vl = inputs.decode(seed=41, S=8192, vl_lo=1000, vl_hi=8192)
-    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
-    outs = [torch.empty((8, 512), dtype=torch.int32, device="cuda") for _ in range(3)]
-    ds.ds_indexer_topk(qd, kd, wd, 512, valid_len=vd, out_idx=outs[0])   # warm-up outside capture
-    torch.cuda.synchronize()
-    gr = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gr):
-        for o in outs:
-            ds.ds_indexer_topk(qd, kd, wd, 512, valid_len=vd, out_idx=o)
-    ref, _ = oracle.indexer_topk(q, kc, w, 512, vl)
-    for _ in range(3):
-        for o in outs:
-            o.fill_(-7)
-        gr.replay()
-        torch.cuda.synchronize()
-        assert ds.ds_get_device_status() == ds.DS_OK
-        for o in outs:
-            check_selection(q, kc, w, vl, 512, o.cpu().numpy(), None)
-
-
-# ---------------------------------------------------------------- row-per-cluster path
-
-@pytest.fixture
-def rowcluster(monkeypatch):
-    # one cluster per row, whatever the batch (the default takes it for small batches)
-    monkeypatch.setenv("DS_INDEXER_ROWCLUSTER", "1")
-
-
-def test_rowcluster_matches_unfused_path(cuda_device, rowcluster, monkeypatch):
-    # both paths compute the float32 scores in the same order (tensor-core dot
-    # products, then the weighted head sum from head 0 up), so they select the
-    # same positions and return the same scores
-    q, kc, w, vl = inputs.decode(seed=37)
-    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
-    got, gs = ds.ds_indexer_topk(qd, kd, wd, 1024, valid_len=vd, return_score=True)
-    torch.cuda.synchronize()
-    monkeypatch.setenv("DS_INDEXER_UNFUSED", "1")
-    ref, rs = ds.ds_indexer_topk(qd, kd, wd, 1024, valid_len=vd, return_score=True)
-    torch.cuda.synchronize()
-    assert ds.ds_get_device_status() == ds.DS_OK
-    g, r = got.cpu().numpy(), ref.cpu().numpy()
-    for t in range(q.shape[0]):
-        assert np.array_equal(np.sort(g[t]), np.sort(r[t])), f"row {t}"
-        og, orr = np.argsort(g[t]), np.argsort(r[t])
-        assert np.array_equal(gs.cpu().numpy()[t][og], rs.cpu().numpy()[t][orr])
-
-
-@pytest.mark.parametrize("B,H,S,k", [(1, 64, 32768, 2048), (16, 64, 32768, 1024), (5, 64, 7000, 512),
-                                     (8, 64, 128, 64), (2, 64, 129, 2048), (3, 40, 20000, 100),
-                                     (4, 64, 300, 1), (20, 64, 5000, 256)])
-def test_rowcluster_shapes(cuda_device, rowcluster, B, H, S, k):
+@pytest.mark.parametrize("B,H,S,k", [(1, 64, 40000, 2048), (5, 64, 7000, 512), (8, 64, 128, 64),
+                                     (2, 64, 75000, 100), (16, 64, 32768, 1024), (2, 64, 129, 2048),
+                                     (3, 40, 20000, 100), (4, 64, 300, 1), (20, 64, 5000, 256),
+                                     (600, 64, 2048, 512), (161, 64, 3001, 2048), (600, 24, 1000, 100), (601, 64, 777, 2048),
+                                     (1, 64, 131072, 2048)])
+def test_fused_shapes(cuda_device, B, H, S, k):
+    # whole-row groups (B >= 148 groups' worth of work, short rows) and split
+    # rows; ragged S, rows longer than one CTA's 16-bit counters (S = 131072:
+    # 1024 tiles over several CTAs), valid_len of 0, negative or past S
     q, kc, w = inputs.indexer_factors(seed=B * 5 + S + H, batch=B, n=S, heads=H)
     g = np.random.default_rng(S + B)
     vl = g.integers(-3, S + 5, size=B).astype(np.int32)
@@ -274,8 +218,9 @@ def test_rowcluster_shapes(cuda_device, rowcluster, B, H, S, k):
     check_selection(q, kc, w, vl, k, idx.cpu().numpy(), score.cpu().numpy())
 
 
-@pytest.mark.parametrize("B,H,S,k", [(8, 64, 32768, 2048), (3, 64, 5000, 1000), (2, 24, 777, 700)])
-def test_rowcluster_exact_arithmetic(cuda_device, rowcluster, B, H, S, k):
+@pytest.mark.parametrize("B,H,S,k", [(8, 64, 32768, 2048), (3, 64, 5000, 1000), (2, 24, 777, 700),
+                                     (640, 64, 1000, 300), (160, 16, 2000, 2048), (600, 16, 300, 50)])
+def test_fused_exact_arithmetic(cuda_device, B, H, S, k):
     # small-integer inputs: exact float32 scores with many equal values, so the
     # index sets must match the oracle's exactly, ties to the lower position
     q, kc, w = exact_inputs(B * 13 + S, B, H, S)
@@ -291,37 +236,41 @@ def test_rowcluster_exact_arithmetic(cuda_device, rowcluster, B, H, S, k):
         assert np.array_equal(score[t, :m].astype(np.float64), ref_scores[t, idx[t, :m]])
 
 
-@pytest.mark.parametrize("S,L", [(32768, 32768), (20000, 12000), (4096, 4000)])
-def test_rowcluster_all_scores_equal(cuda_device, rowcluster, S, L):
-    # zero weights: every score is 0, the whole row sits in one radix bin (past
-    # the leader's list capacity for the longest rows) and the k lowest
+@pytest.mark.parametrize("B,S,L", [(2, 32768, 32768), (2, 20000, 12000), (2, 4096, 4000), (600, 2000, 2000)])
+def test_fused_all_scores_equal(cuda_device, B, S, L):
+    # zero weights: every score is 0, the whole row sits in one histogram bin
+    # (past the candidate list's capacity for the longest rows) and the k lowest
     # positions must be returned
-    q, kc, w = inputs.indexer_factors(seed=S, batch=2, n=S, heads=64)
+    q, kc, w = inputs.indexer_factors(seed=S, batch=B, n=S, heads=64)
     w = np.zeros_like(w)
-    vl = np.array([L, L // 3], dtype=np.int32)
+    vl = np.full(B, L, dtype=np.int32)
+    vl[1] = L // 3
     qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
     idx, score = ds.ds_indexer_topk(qd, kd, wd, 2048, valid_len=vd, return_score=True)
     torch.cuda.synchronize()
     assert ds.ds_get_device_status() == ds.DS_OK
     idx = idx.cpu().numpy()
-    for t in range(2):
+    for t in range(B):
         m = min(2048, int(vl[t]))
         assert np.array_equal(np.sort(idx[t, :m]), np.arange(m)), f"row {t}"
         assert np.all(idx[t, m:] == -1)
-    assert np.all(score.cpu().numpy()[:, :min(2048, L // 3)] == 0.0)
+    assert np.all(score.cpu().numpy()[1, :min(2048, L // 3)] == 0.0)
 
 
-def test_rowcluster_graph_replay(cuda_device, rowcluster):
-    q, kc, w, vl = inputs.decode(seed=43, S=8192, vl_lo=1000, vl_hi=8192)
+@pytest.mark.parametrize("B", [8, 600])
+def test_fused_graph_replay(cuda_device, B):
+    # the split-row path leaves its histograms and tickets zero for the next
+    # launch; replaying a graph of 3 calls several times must keep results right
+    q, kc, w, vl = inputs.decode(seed=43, batch=B, S=8192, vl_lo=1000, vl_hi=8192)
     qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
-    outs = [torch.empty((8, 512), dtype=torch.int32, device="cuda") for _ in range(3)]
-    ds.ds_indexer_topk(qd, kd, wd, 512, valid_len=vd, out_idx=outs[0])
+    outs = [torch.empty((B, 512), dtype=torch.int32, device="cuda") for _ in range(3)]
+    ds.ds_indexer_topk(qd, kd, wd, 512, valid_len=vd, out_idx=outs[0])   # warm-up outside capture
     torch.cuda.synchronize()
     gr = torch.cuda.CUDAGraph()
     with torch.cuda.graph(gr):
         for o in outs:
             ds.ds_indexer_topk(qd, kd, wd, 512, valid_len=vd, out_idx=o)
-    for _ in range(2):
+    for _ in range(3):
         for o in outs:
             o.fill_(-7)
         gr.replay()
