@@ -41,9 +41,10 @@
  *    equal.  Positions s >= valid_len[row] are never selected.  When a row
  *    has fewer than k eligible positions, the missing slots hold index -1 and
  *    value / score -inf.
- *  - The library owns only scratch memory: ds_indexer_topk and
- *    ds_sparse_attention each allocate a per-device, grow-only buffer with
- *    cudaMalloc on first use (so make the first call outside CUDA-graph
+ *  - The library owns only scratch memory: ds_indexer_topk (score rows and
+ *    per-row key histograms) and ds_sparse_attention each allocate
+ *    per-device, grow-only buffers with cudaMalloc on first use and on calls
+ *    larger than any before (so make those calls outside CUDA-graph
  *    capture); ds_release frees them.
  *  - Calls on different streams may run concurrently, except that calls of
  *    ds_indexer_topk on one device share the scratch buffer and must be
@@ -130,8 +131,14 @@ int ds_indexer_score(const void* q, const void* kcache, const float* w,
 /*
  * ds_indexer_topk -- indexer score followed by the top-k positions of each row.
  *   (NKI pull request "Add DeepSeek-V4 CSA attention kernels", steps table
- *    rows 2 and 3, and "The top-k on the GPSIMD engine": scoring fused with
- *    the selection so that the score row does not go back in full.)
+ *    rows 2 and 3, and "The top-k on the GPSIMD engine": the scores feed the
+ *    top-k as they are produced.)
+ *
+ * When a row is scored by several CTAs (few rows, as in decode) the scorer
+ * also counts every score in an exact per-row histogram of its key's top 12
+ * bits, and the selection starts from the threshold bin those counts give;
+ * with many rows the scores go to the scratch buffer and ds_topk's kernel
+ * selects them.  The result is the same either way.
  *
  * q, kcache, w, batch, heads, d, S, valid_len  as for ds_indexer_score.
  * k          1 <= k <= DS_MAX_K.
@@ -162,8 +169,7 @@ int ds_indexer_topk(const void* q, const void* kcache, const float* w,
  * sorted_index 0 or 1: with 1 each row's selection is in ascending position
  *            order (the selection itself is the same).
  * The other arguments, outputs and results are those of ds_indexer_topk,
- * including its use of the scratch buffer; this entry point always runs the
- * scorer and the top-k as two launches.
+ * including its use of the scratch buffer and its choice of selection.
  */
 int ds_indexer_topk_ex(const void* q, const void* kcache, int64_t kcache_batch_stride, const float* w,
                        int batch, int heads, int d, int S, const int32_t* valid_len, int k,
