@@ -196,7 +196,7 @@ static cudaError_t launch_topk(const TopkParams& p, int C, cudaStream_t st) {
 // idle and every slice keeps at least 32768 scores.
 static int topk_stash_enqueue(const void* scores, int batch, int n, int k, int dtype, const int32_t* valid_len,
                               int32_t* out_idx, void* out_val, int return_value, int sorted_index,
-                              cudaStream_t st, DeviceState* s) {
+                              cudaStream_t st, DeviceState* s, uint32_t* ghist = nullptr) {
   if (n > kMaxRowElems) return DS_ERR_ARG;
   int C = 1;
   const char* force = getenv("DS_TOPK_CLUSTER");  // tuning sweeps only
@@ -209,7 +209,9 @@ static int topk_stash_enqueue(const void* scores, int batch, int n, int k, int d
   int slice = (n + C - 1) / C;
   slice = (slice + 7) / 8 * 8;
   TsParams p;
+  memset(&p, 0, sizeof(p));
   p.scores = scores;
+  p.ghist = dtype == DS_F32 ? ghist : nullptr;
   p.valid_len = valid_len;
   p.out_idx = out_idx;
   p.out_val = out_val;
@@ -482,14 +484,14 @@ static void* get_scratch(DeviceState* s, size_t bytes) {
 
 // ---- indexer + top-k (the path of ds_indexer_topk and ds_indexer_topk_ex)
 //
-// Rows split over several scorer CTAs (few rows, as in decode): the scorer
-// also counts every valid score in an exact histogram of its key's top 12 bits
-// (per row, added into global memory), and topk_hist_select_kernel starts from
-// the threshold bin those counts give: no sampling and no histogram pass of
-// its own.  Whole rows per scorer CTA (many rows, as in prefill): the scores
-// go to the [B, S] buffer and ds_topk's kernel selects them; on this GPU that
-// measured faster than selecting inside the scorer's CTAs (whose selection
-// tail leaves the tensor pipe idle) or beside them.
+// The scorer also counts every valid score in an exact histogram of its key's
+// top 12 bits (per row, added into global memory), and the selection starts
+// from the threshold bin those counts give, with no sampling.  Rows split over
+// several scorer CTAs (few rows, as in decode): topk_hist_select_kernel, a
+// cluster per row.  Whole rows per scorer CTA (many rows, as in prefill): the
+// one-pass stash kernel streams each row once and stashes what is at or above
+// the bin.  Selecting inside the scorer's CTAs (whose selection tail leaves the
+// tensor pipe idle) or beside them measured slower on this GPU.
 
 // Grow-only buffer that is all zero whenever no call is in flight: zeroed when
 // (re)allocated, and every launch that uses it leaves it zero again.
@@ -615,9 +617,12 @@ static int indexer_topk_rows(const void* q, const void* kc, const float* w, int 
     if (rc != DS_OK) return rc;
     return launch_hist_select(sc, gh, vl, out_idx, out_score, B, S, k, sorted, st, s);
   }
-  const int rc = score_enqueue(q, kc, w, B, H, S, vl, sc, st, s, kstride);
+  // whole rows: the scorer's counts give the stash kernel its threshold
+  uint32_t* gh = static_cast<uint32_t*>(get_zeroed_state(s, (size_t)B * kSelBins * sizeof(uint32_t)));
+  if (!gh) return DS_ERR_NOMEM;
+  const int rc = launch_score_hist<NT, HP, ST>(q, kc, w, B, H, S, vl, kstride, sc, gh, st, s);
   if (rc != DS_OK) return rc;
-  return topk_enqueue(sc, B, S, k, DS_F32, vl, out_idx, out_score, out_score != nullptr, sorted, st, s);
+  return topk_stash_enqueue(sc, B, S, k, DS_F32, vl, out_idx, out_score, out_score != nullptr, sorted, st, s, gh);
 }
 
 // Rows per CTA group: as for the scores alone (two rows for 2 and 5..8 rows,

@@ -26,6 +26,11 @@
 //    equal keys) re-reads its slice from L2 and finds its exact k-th (key,
 //    position) with radix passes over the slice, then stashes exactly that
 //    many.
+//  * Rows whose scorer counted them (float32 rows of ds_indexer_topk with an
+//    exact histogram of their keys' top 12 bits) skip the sample: the
+//    threshold is the lower edge of the bin that holds the row's k-th key, so
+//    the union of the stashes is complete by construction and only the
+//    stash's capacity is checked.
 #pragma once
 
 #include "ptx.cuh"
@@ -43,6 +48,7 @@ constexpr int kTsMaxCluster = 4;
 
 struct TsParams {
   const void* scores;
+  uint32_t* ghist;   // float32 rows: [batch, 4096] exact key histograms, or null (cleared here after use)
   const int32_t* valid_len;
   int32_t* out_idx;
   void* out_val;
@@ -381,7 +387,8 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   constexpr int SW = kTsSample / K::kVec;
   constexpr int SPT = (SW + NT - 1) / NT;
   constexpr int kRuns = 64;
-  const bool sampled = m > kTsCap;
+  const bool counted = K::kBits == 32 && p.ghist != nullptr;  // the threshold comes from the row's histogram
+  const bool sampled = !counted && m > kTsCap;
   const int run_w = sampled ? min(nfull, SW) / kRuns : 0;  // >= 7: a sampled slice has > 4096 scores
   const int sw = kRuns * run_w;                            // sampled words, <= nfull
   uint4 s[SPT];
@@ -415,9 +422,21 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   };
 
   // ---- threshold: the sample's key of rank rk, which leaves an expected
-  // need + 4 standard deviations + 8 keys of the slice above it
+  // need + 4 standard deviations + 8 keys of the slice above it.  For float32
+  // keys the lower edge of its 12-bit bin is close enough (a second digit
+  // pass costs more than the few extra keys stashed); for bfloat16 keys, with
+  // only 4 bits below the first digit, the second digit keeps the stash small.
   uint32_t t = 0u;
-  if (sampled) {
+  if (counted) {
+    // the bin of the row's kk-th key from the scorer's counts
+    const uint4* gh = reinterpret_cast<const uint4*>(p.ghist + (size_t)row * 4096);
+    for (int i = tid; i < 1024; i += NT) reinterpret_cast<uint4*>(shist)[i] = __ldcg(gh + i);
+    for (int st = 0; st < kTsStages - 1; ++st) issue(st);
+    __syncthreads();
+    uint32_t above, inbin;
+    const uint32_t b0 = ts_find_bin<NT>(shist, 4096, (uint32_t)kk, ctrl, above, inbin);
+    t = b0 << kShift0;
+  } else if (sampled) {
     for (int i = tid; i < 4096; i += NT) shist[i] = 0u;
     __syncthreads();
 #pragma unroll
@@ -434,6 +453,9 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
     const int rk = min(ns, (int)ceilf(lam + 4.0f * sqrtf(lam) + 8.0f));
     uint32_t above, inbin;
     const uint32_t b1 = ts_find_bin<NT>(shist, 4096, (uint32_t)rk, ctrl, above, inbin);
+    if constexpr (K::kBits == 32) {
+      t = b1 << kShift0;
+    } else {
     constexpr int W2 = kShift0 >= 11 ? 11 : kShift0;
     constexpr int SH2 = kShift0 - W2;
     for (int i = tid; i < (1 << W2); i += NT) shist[i] = 0u;
@@ -452,6 +474,7 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
     uint32_t a2, i2;
     const uint32_t b2 = ts_find_bin<NT>(shist, 1 << W2, (uint32_t)(rk - (int)above), ctrl, a2, i2);
     t = ((b1 << W2) | b2) << SH2;
+    }
   } else {
     for (int st = 0; st < kTsStages - 1; ++st) issue(st);
     __syncthreads();  // the zeroed histogram and counters
@@ -528,7 +551,7 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   };
 
   uint32_t cnt = ctrl->cnt;
-  const bool ok = cnt >= (uint32_t)need && cnt <= (uint32_t)kTsCap;
+  const bool ok = (counted || cnt >= (uint32_t)need) && cnt <= (uint32_t)kTsCap;
   bool all_ok = ok;
   if (C > 1) {
     cluster_sync();  // every CTA has streamed: the leader's ring is free
@@ -538,6 +561,12 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
     for (int c = 0; c < C; ++c) all_ok &= ctrl->ok[c] != 0u;
   }
   if (tid == 0 && crank == 0) ctrl->tab[0] = cnt;
+  // every CTA of the row has read the row's counts: the leader clears them
+  // for the next call
+  if (counted && crank == 0) {
+    uint4* gh = reinterpret_cast<uint4*>(p.ghist + (size_t)row * 4096);
+    for (int i = tid; i < 1024; i += NT) gh[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
 
   if (!all_ok) {
     // ---- exact fallback (uniform decision; only CTAs with a bad stash work):
