@@ -36,6 +36,8 @@
  *    errors are detected on the host before anything is enqueued.  Errors
  *    found on the device (a bounded wait that ran out) are recorded in a
  *    per-device status word that ds_get_device_status reads and clears.
+ *    libdstopk_debug.so, the same library built with DS_DEBUG, also records
+ *    inputs read on the device outside their documented range there.
  *  - Index outputs are int32.  Ties between equal scores go to the lower
  *    position; -0.0 equals +0.0; every NaN ranks above +inf and all NaNs are
  *    equal.  Positions s >= valid_len[row] are never selected.  When a row
@@ -69,6 +71,8 @@ typedef enum { DS_F32 = 0, DS_BF16 = 1 } ds_dtype;
 #define DS_ERR_TIMEOUT (-3)     /* a bounded wait inside a kernel ran out (device status) */
 #define DS_ERR_UNSUPPORTED (-4) /* the current device is not an sm_100 GPU */
 #define DS_ERR_NOMEM (-5)       /* the scratch buffer could not be allocated */
+#define DS_ERR_RANGE (-6)       /* DS_DEBUG builds: an input read on the device was out of
+                                   range (device status) */
 
 /* limits */
 #define DS_MAX_K 2048            /* largest k of either operation */
@@ -319,12 +323,47 @@ int ds_sparse_attention(const void* q, const void* kv, int64_t kv_batch_stride, 
 
 /*
  * ds_get_device_status -- synchronise `stream`, then return and clear the
- * current device's status word: DS_OK, or DS_ERR_TIMEOUT if a kernel's bounded
- * wait ran out since the last call (its outputs are then unspecified), or
- * DS_ERR_CUDA if the synchronisation itself failed.
+ * current device's status word: DS_OK; DS_ERR_TIMEOUT if a kernel's bounded
+ * wait ran out since the last call (the outputs of that call are then
+ * unspecified, but every index is -1 or a valid position); DS_ERR_RANGE
+ * (libdstopk_debug.so only) if a kernel read an input outside its documented
+ * range -- a valid_len outside [0, n], an attention slot other than -1
+ * outside [0, T), a win_len outside [0, W] -- which it then clamped or skipped
+ * exactly as the release build does; or DS_ERR_CUDA if the synchronisation
+ * itself failed.  The first error recorded since the last call is the one
+ * returned.
  * (No counterpart on the pages: the library's error reporting.)
  */
 int ds_get_device_status(void* stream);
+
+/*
+ * ds_set_wait_limit -- the limit of every bounded wait inside the kernels
+ * (an mbarrier wait for a copy, a tensor-core result or a peer CTA), in
+ * nanoseconds of the GPU's global timer: 0 restores the default of one
+ * second; 0 <= ns <= 60 s, else DS_ERR_ARG.  Read by every launch enqueued
+ * after the call (a CUDA graph keeps the limit it was captured with).  A wait
+ * that runs out records DS_ERR_TIMEOUT and lets its kernel finish.
+ * (No counterpart on the pages: the library's failure detection.)
+ */
+int ds_set_wait_limit(int64_t ns);
+
+/*
+ * ds_plant_wait_fault -- testing the failure detection: the next `launches`
+ * indexer scorer launches (of ds_indexer_score, ds_indexer_topk and its
+ * variants) each carry a planted fault: in their first CTA one epilogue warp
+ * skips its first release of a tensor-core accumulator, so that the MMA warp's
+ * wait for that accumulator, and the waits behind it, run out after the wait
+ * limit.  The kernel then scores that CTA's remaining positions as -inf, lets
+ * its copies in flight land, frees its tensor memory and returns; the call's
+ * status is DS_ERR_TIMEOUT.  0 disarms.  launches >= 0, else DS_ERR_ARG.
+ * Nothing traps, and the next call without the fault runs normally.
+ * (No counterpart on the pages.)
+ */
+int ds_plant_wait_fault(int launches);
+
+/* ds_debug_build -- 1 in libdstopk_debug.so (compiled with DS_DEBUG: device
+ * range checks that record DS_ERR_RANGE), 0 in libdstopk.so. */
+int ds_debug_build(void);
 
 /* ds_strerror -- a static, human-readable name for a status code. */
 const char* ds_strerror(int code);

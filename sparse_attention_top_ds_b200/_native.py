@@ -8,8 +8,10 @@ fallback implementation.
 import ctypes
 import os
 
-_LIB_PATH = os.environ.get(
-    "DS_TOPK_LIB", os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdstopk.so"))
+_PKG = os.path.dirname(os.path.abspath(__file__))
+# DS_TOPK_LIB may name another build, such as libdstopk_debug.so (device range checks)
+_LIB_PATH = os.environ.get("DS_TOPK_LIB", os.path.join(_PKG, "libdstopk.so"))
+DEBUG_LIB_PATH = os.path.join(_PKG, "libdstopk_debug.so")
 
 DS_F32 = 0
 DS_BF16 = 1
@@ -20,6 +22,7 @@ DS_ERR_CUDA = -2
 DS_ERR_TIMEOUT = -3
 DS_ERR_UNSUPPORTED = -4
 DS_ERR_NOMEM = -5
+DS_ERR_RANGE = -6
 
 DS_MAX_K = 2048
 DS_INDEXER_DIM = 128
@@ -75,6 +78,12 @@ def load():
     lib.ds_strerror.restype = ctypes.c_char_p
     lib.ds_release.argtypes = []
     lib.ds_release.restype = None
+    lib.ds_set_wait_limit.argtypes = [ctypes.c_int64]
+    lib.ds_set_wait_limit.restype = i32
+    lib.ds_plant_wait_fault.argtypes = [i32]
+    lib.ds_plant_wait_fault.restype = i32
+    lib.ds_debug_build.argtypes = []
+    lib.ds_debug_build.restype = i32
     _lib = lib
     return lib
 
@@ -125,6 +134,22 @@ def ds_get_device_status(stream=None):
 
 def ds_release():
     load().ds_release()
+
+
+def ds_set_wait_limit(ns):
+    """Limit of the kernels' bounded waits in ns (0: the default of one second)."""
+    _check(load().ds_set_wait_limit(int(ns)), "ds_set_wait_limit")
+
+
+def ds_plant_wait_fault(launches):
+    """Testing the failure detection: the next `launches` scorer launches each
+    make one of their bounded waits run out (DS_ERR_TIMEOUT in the status)."""
+    _check(load().ds_plant_wait_fault(int(launches)), "ds_plant_wait_fault")
+
+
+def ds_debug_build():
+    """True for the DS_DEBUG build (device range checks -> DS_ERR_RANGE)."""
+    return bool(load().ds_debug_build())
 
 
 # ------------------------------------------------------------------ torch-tensor front end

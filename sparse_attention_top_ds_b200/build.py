@@ -1,4 +1,6 @@
-"""Build libdstopk.so in-tree for sm_100a with nvcc (no JIT cache).
+"""Build libdstopk.so in-tree for sm_100a with nvcc (no JIT cache), and next
+to it libdstopk_debug.so, the same library compiled with DS_DEBUG (device range
+checks that record DS_ERR_RANGE in the status word).
 
     python -m sparse_attention_top_ds_b200.build          # build if stale
     python -m sparse_attention_top_ds_b200.build --force  # always rebuild
@@ -14,6 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 HEADER = os.path.join(ROOT, "include", "ds_topk.h")
 LIB = os.path.join(PKG, "libdstopk.so")
+LIB_DEBUG = os.path.join(PKG, "libdstopk_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -40,25 +43,35 @@ def sources():
     return files
 
 
-def stale():
-    if not os.path.exists(LIB):
+def stale(lib=LIB):
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(f) > t for f in sources())
 
 
 def build(force=False, verbose=False):
-    """Compile csrc/lib.cu into libdstopk.so next to this file; return its path."""
-    if not force and not stale():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [nvcc_path()] + NVCC_FLAGS + ["-o", tmp, os.path.join(CSRC, "lib.cu")]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    if res.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
-    os.replace(tmp, LIB)
+    """Compile csrc/lib.cu into libdstopk.so and libdstopk_debug.so next to
+    this file (the two nvcc runs side by side); return the release path."""
+    jobs = []
+    for lib, extra in ((LIB, []), (LIB_DEBUG, ["-DDS_DEBUG"])):
+        if not force and not stale(lib):
+            continue
+        tmp = lib + ".tmp"
+        cmd = [nvcc_path()] + NVCC_FLAGS + extra + ["-o", tmp, os.path.join(CSRC, "lib.cu")]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+        jobs.append((lib, tmp, proc))
+    errors = []
+    for lib, tmp, proc in jobs:
+        out, err = proc.communicate()
+        if proc.returncode != 0:
+            errors.append(f"nvcc failed for {os.path.basename(lib)}:\n" + out + err)
+        else:
+            os.replace(tmp, lib)
+    if errors:
+        raise RuntimeError("\n".join(errors))
     return LIB
 
 

@@ -60,6 +60,7 @@ struct AttnParams {
   uint16_t* out;           // bf16 [B, H, D]
   float* lse;              // [B, H] or null
   int* status;
+  uint64_t wait_ns;        // limit of every bounded wait (0: the library default)
   int T, k, W, B, H, D, HT, NS;
   float scale_log2;        // scale * log2(e)
 };
@@ -68,9 +69,11 @@ struct AttnParams {
 __device__ __forceinline__ const uint16_t* attn_row_src(const AttnParams& p, int b, int j) {
   if (j < p.k) {
     const int r = p.idx[(size_t)b * p.k + j];
+    debug_range(r >= -1 && r < p.T, p.status);
     if (r >= 0 && r < p.T) return p.kv + (long long)b * p.kv_bstride + (long long)r * p.D;
   } else if (j < p.k + p.W) {
     int wl = p.win_len ? p.win_len[b] : p.W;
+    debug_range(wl >= 0 && wl <= p.W, p.status);
     wl = wl < 0 ? 0 : (wl > p.W ? p.W : wl);
     const int i = j - p.k;
     if (i < wl) return p.win + ((long long)b * p.W + i) * p.D;
@@ -186,7 +189,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   // ---- S = Q . R^T into TMEM columns [0, 64)
   if (tid == 0) {
-    const bool ok = mbar_wait_bounded(bar_q, 0, p.status);
+    const bool ok = mbar_wait_bounded(bar_q, 0, p.status, p.wait_ns);
     tc_fence_after();
     if (ok) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, kAttnRows);
@@ -214,7 +217,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int half = warp >> 2;
     const int h = (warp & 3) * 32 + lane;
     float* xch = reinterpret_cast<float*>(smem + AttnSmem::kv_off(D));  // the row tiles are no longer read
-    mbar_wait_bounded(bar_s, 0, p.status);
+    mbar_wait_bounded(bar_s, 0, p.status, p.wait_ns);
     __syncwarp();
     tc_fence_after();
     const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(half * 32);
@@ -383,7 +386,8 @@ __global__ void __launch_bounds__(kPvWarps * 32, 1) sparse_attn_pv_kernel(const 
       for (int j = 0; j < nstage; ++j) {
         const int s = j % kPvStages;
         const int c = c0 + j * K, n = min(K, c0 + nmine - c);
-        if (j >= kPvStages) mbar_wait_bounded(empty0 + 8u * s, (uint32_t)((j / kPvStages - 1) & 1), p.status);
+        if (j >= kPvStages)
+          mbar_wait_bounded(empty0 + 8u * s, (uint32_t)((j / kPvStages - 1) & 1), p.status, p.wait_ns);
         const uint32_t st = sbase + (uint32_t)s * L_::kStage;
         mbar_arrive_expect_tx(full0 + 8u * s, (uint32_t)n * (kAttnTile + kRowTile));
         bulk_g2s(st, p.ptile + (row0 + c) * (size_t)kAttnTile, (uint32_t)n * kAttnTile, full0 + 8u * s);
@@ -399,7 +403,7 @@ __global__ void __launch_bounds__(kPvWarps * 32, 1) sparse_attn_pv_kernel(const 
     const int hg = ht * kAttnHeads + h;
     const float sink_l2 = (p.sink && hg < p.H) ? p.sink[hg] * kLog2e : -INFINITY;
     M = sink_l2;
-    if (NS > 0) mbar_wait_bounded(bar_ml, 0, p.status);
+    if (NS > 0) mbar_wait_bounded(bar_ml, 0, p.status, p.wait_ns);
     for (int c = 0; c < NS; ++c) {
       const float2 v = ml_s[c * kAttnHeads + h];
       if (v.y > 0.0f) M = fmaxf(M, v.x);
@@ -413,7 +417,7 @@ __global__ void __launch_bounds__(kPvWarps * 32, 1) sparse_attn_pv_kernel(const 
     for (int j = 0; j < nstage; ++j) {
       const int s = j % kPvStages;
       const int c = c0 + j * K, n = min(K, c0 + nmine - c);
-      mbar_wait_bounded(full0 + 8u * s, (uint32_t)((j / kPvStages) & 1), p.status);
+      mbar_wait_bounded(full0 + 8u * s, (uint32_t)((j / kPvStages) & 1), p.status, p.wait_ns);
       for (int t = 0; t < n; ++t) {
         const float2 v = ml_s[(c + t) * kAttnHeads + h];
         const float f = v.y > 0.0f ? exp2f(v.x - M) * invL : 0.0f;
@@ -438,7 +442,7 @@ __global__ void __launch_bounds__(kPvWarps * 32, 1) sparse_attn_pv_kernel(const 
     for (int j = 0; j < nstage; ++j) {
       const int s = j % kPvStages;
       const int n = min(K, c0 + nmine - (c0 + j * K));
-      mbar_wait_bounded(ready0 + 8u * s, (uint32_t)((j / kPvStages) & 1), p.status);
+      mbar_wait_bounded(ready0 + 8u * s, (uint32_t)((j / kPvStages) & 1), p.status, p.wait_ns);
       fence_proxy_async_smem();
       tc_fence_after();
       const uint32_t st = sbase + (uint32_t)s * L_::kStage;
@@ -458,7 +462,7 @@ __global__ void __launch_bounds__(kPvWarps * 32, 1) sparse_attn_pv_kernel(const 
   if (warp >= 1 && warp <= 8) {
     uint32_t r[32];
     if (nmine > 0) {
-      mbar_wait_bounded(bar_done, 0, p.status);
+      mbar_wait_bounded(bar_done, 0, p.status, p.wait_ns);
       __syncwarp();
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(half * 32);
@@ -487,7 +491,7 @@ __global__ void __launch_bounds__(kPvWarps * 32, 1) sparse_attn_pv_kernel(const 
                        : "memory");
       } else {
         if (h == 0) mbar_arrive_expect_tx(bar_recv, kAttnHeads * 32 * 4);  // 128 heads x 32 columns from the partner
-        mbar_wait_bounded(bar_recv, 0, p.status);
+        mbar_wait_bounded(bar_recv, 0, p.status, p.wait_ns);
         if (hg < p.H) pv_emit<true>(r, recv + h * 32, h & 7, orow);
       }
     } else if (hg < p.H) {

@@ -57,6 +57,9 @@ struct ScoreParams {
   int ctas_per_group;       // CTAs sharing one group of NT rows
   int key_per_row;          // 1: row t reads key cache t (then NT == 1); 0: one cache for every row
   uint32_t* ghist;          // SEL: [B, 4096] key histograms, zero before the launch
+  uint64_t wait_ns;         // limit of every bounded wait (0: the library default)
+  int fault;                // testing the failure detection: 1 = CTA 0's first epilogue warp skips its
+                            // first release of the accumulator, so that a wait runs out (0 otherwise)
 };
 
 template <int NT, int HP, int STAGES, bool SEL = false>
@@ -80,6 +83,7 @@ struct ScoreCfg {
   static constexpr int kOffHist = kOffW + NT * HP * 4;          // SEL: u16 key histograms, 2 per word
   static constexpr int kHistBytes = SEL ? NT * (kSelBins / 2) * 4 : 0;
   static constexpr int kOffBar = kOffHist + kHistBytes;
+  // (tiles whose key loads the MMA warp has waited for: the drain at the end)
   // barriers: qfull, kfull[STAGES], kempty[STAGES], afull[2], aempty[2], tmem slot
   static constexpr int kBarQ = 0;
   static constexpr int kBarKFull = 1;
@@ -88,6 +92,7 @@ struct ScoreCfg {
   static constexpr int kBarAEmpty = 3 + 2 * STAGES;
   static constexpr int kNumBars = 5 + 2 * STAGES;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+  static constexpr int kOffConsumed = kOffTmemSlot + 8;
   static constexpr int kSmemBytes = kOffTmemSlot + 16 + 1024;  // + alignment slack
   static_assert(kN % 16 == 0 && kN <= 256 && kN % kNmma == 0, "bad tile");
   static_assert(HP % 16 == 0 && HP <= 64, "bad head padding");
@@ -129,6 +134,7 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES, SEL>::kThreads, 1)
   for (int t = 0; t < NT; ++t) {
     if (t0 + t < p.B) {
       int v = p.valid_len ? p.valid_len[t0 + t] : p.S;
+      if (threadIdx.x == 0 && blockIdx.x % p.ctas_per_group == 0) debug_range(v >= 0 && v <= p.S, p.status);
       v = v < 0 ? 0 : (v > p.S ? p.S : v);
       maxvl = max(maxvl, v);
     }
@@ -178,30 +184,37 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES, SEL>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  uint32_t* consumed = reinterpret_cast<uint32_t*>(smem + C::kOffConsumed);  // [0] tiles, [1] queries
+  const uint64_t wait_ns = p.wait_ns;
+  int issued = min(nact, STAGES);  // thread 0: key tiles whose loads are issued
   if (warp == 0) {
     // ---------------- TMA producer
     if (lane == 0 && nact > 0) {
       for (int i = STAGES; i < nact; ++i) {
         const int s = i % STAGES, r = i / STAGES;
-        if (!mbar_wait_bounded(BAR(C::kBarKEmpty + s), (r & 1) ^ 1, p.status)) break;
+        if (!mbar_wait_bounded(BAR(C::kBarKEmpty + s), (r & 1) ^ 1, p.status, wait_ns)) break;
         const int pos0 = (tile_lo + i) * 128;
         mbar_arrive_expect_tx(BAR(C::kBarKFull + s), C::kStage);
         tma_load_4d(sbase + C::kOffK + s * C::kStage, &tm_k, 0, pos0, 0, kcache, BAR(C::kBarKFull + s));
+        issued = i + 1;
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0 && nact > 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, C::kNmma);
-      bool ok = mbar_wait_bounded(BAR(C::kBarQ), 0, p.status);
+      bool ok = mbar_wait_bounded(BAR(C::kBarQ), 0, p.status, wait_ns);
+      consumed[1] = ok ? 1u : 0u;
+      consumed[0] = 0u;
       for (int i = 0; i < nact && ok; ++i) {
         const int s = i % STAGES, r = i / STAGES;
-        if (!mbar_wait_bounded(BAR(C::kBarKFull + s), r & 1, p.status)) break;
+        if (!mbar_wait_bounded(BAR(C::kBarKFull + s), r & 1, p.status, wait_ns)) break;
+        consumed[0] = (uint32_t)(i + 1);
         const uint32_t a_base = sbase + C::kOffK + s * C::kStage;
         // the whole tile in accumulator buffer i % 2
         const int slot = i % C::kNbuf;
         const int use = i / C::kNbuf;
-        if (!mbar_wait_bounded(BAR(C::kBarAEmpty + slot), (use & 1) ^ 1, p.status)) break;
+        if (!mbar_wait_bounded(BAR(C::kBarAEmpty + slot), (use & 1) ^ 1, p.status, wait_ns)) break;
         tc_fence_after();
         const uint32_t d_base = tmem_base + (uint32_t)(slot * C::kN);
 #pragma unroll
@@ -240,11 +253,15 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES, SEL>::kThreads, 1)
       }
       vl[j] = v;
     }
+    int done = nact;  // tiles scored: fewer once a wait has run out
     for (int i = 0; i < nact; ++i) {
       const int b = i % C::kNbuf;  // TMEM buffer of this tile
       const int slot = b;
       const int u = i / C::kNbuf;
-      if (!mbar_wait_bounded(BAR(C::kBarAFull + slot), u & 1, p.status)) break;  // status records the timeout
+      if (!mbar_wait_bounded(BAR(C::kBarAFull + slot), u & 1, p.status, wait_ns)) {  // status records it
+        done = i;
+        break;
+      }
       tc_fence_after();
       const int s = (tile_lo + i) * 128 + row;
 #pragma unroll
@@ -273,11 +290,31 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES, SEL>::kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C::kBarAEmpty + slot));
+      // (testing the failure detection: CTA 0's first epilogue warp may skip
+      // its first release, so that the MMA warp's wait for this buffer runs out)
+      const bool skip = p.fault == 1 && blockIdx.x == 0 && e == 0 && i == 0;
+      if (lane == 0 && !skip) mbar_arrive(BAR(C::kBarAEmpty + slot));
     }
-    // tiles past the group's valid lengths: no products, -inf (the selection
-    // never reads them)
-    for (int tile = act_hi > tile_lo ? act_hi : tile_lo; !SEL && tile < tile_hi; ++tile) {
+    // after a wait that ran out, the valid positions left still get a score:
+    // -inf (counted too), so that the rows and their histograms stay in step
+    if constexpr (SEL) {
+      const uint32_t bin_ninf = F32Keys::key(__float_as_uint(-INFINITY)) >> kSelShift;
+      for (int i = done; i < nact; ++i) {
+        const int s = (tile_lo + i) * 128 + row;
+#pragma unroll
+        for (int j = 0; j < TPH; ++j) {
+          const int tl = hf * TPH + j;
+          const int t = t0 + tl;
+          if (tl < NT && t < p.B && s < vl[j]) {
+            atomicAdd(hist16 + tl * (kSelBins / 2) + (bin_ninf >> 1), 1u << ((bin_ninf & 1u) << 4));
+            p.out[(size_t)t * p.S + s] = -INFINITY;
+          }
+        }
+      }
+    }
+    // tiles past the group's valid lengths (and, after a wait that ran out,
+    // the tiles left): no products, -inf (the selection never reads them)
+    for (int tile = tile_lo + done; !SEL && tile < tile_hi; ++tile) {
       const int s = tile * 128 + row;
 #pragma unroll
       for (int j = 0; j < TPH; ++j) {
@@ -291,6 +328,13 @@ __global__ void __launch_bounds__(ScoreCfg<NT, HP, STAGES, SEL>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // after a wait that ran out, key tiles (or the queries) may still be on
+  // their way into shared memory: wait for them (bounded) before the CTA ends
+  if (threadIdx.x == 0 && nact > 0) {
+    if (consumed[1] == 0u) mbar_wait_bounded(BAR(C::kBarQ), 0, p.status, wait_ns);
+    for (int j = (int)consumed[0]; j < issued; ++j)
+      mbar_wait_bounded(BAR(C::kBarKFull + j % STAGES), (uint32_t)((j / STAGES) & 1), p.status, wait_ns);
+  }
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
   if constexpr (SEL) {
     // every score is counted: add this CTA's counts into the rows' global

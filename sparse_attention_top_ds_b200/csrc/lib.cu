@@ -2,6 +2,7 @@
 // argument checks, launch-shape choice and kernel launches.  One translation
 // unit holds every kernel, so device symbols (the status word) resolve here.
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -42,6 +43,21 @@ struct DeviceState {
 
 static std::mutex g_mu;
 static DeviceState g_dev[kMaxDevices];
+
+// Limit of the kernels' bounded waits, in ns (0: kWaitLimitNs), read at each
+// launch; and the number of scorer launches still to carry the planted fault
+// that makes one of their waits run out (testing the failure detection).
+static std::atomic<long long> g_wait_ns{0};
+static std::atomic<int> g_planted{0};
+
+static uint64_t wait_limit() { return (uint64_t)g_wait_ns.load(std::memory_order_relaxed); }
+
+static int take_planted_fault() {
+  int n = g_planted.load(std::memory_order_relaxed);
+  while (n > 0 && !g_planted.compare_exchange_weak(n, n - 1, std::memory_order_relaxed)) {
+  }
+  return n > 0 ? 1 : 0;
+}
 
 static cudaError_t indexer_setup();
 template <int NT>
@@ -221,6 +237,7 @@ static int topk_stash_enqueue(const void* scores, int batch, int n, int k, int d
   p.slice = slice;
   p.return_value = return_value ? 1 : 0;
   p.sorted = sorted_index ? 1 : 0;
+  p.status = s->status;
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)(batch * C), 1, 1);
@@ -405,6 +422,7 @@ static int launch_score(const void* q, const void* kc, const float* w, int B, in
   if (tpc > ntiles) tpc = ntiles;
   const int cpg = (int)((ntiles + tpc - 1) / tpc);
   ScoreParams p;
+  memset(&p, 0, sizeof(p));
   p.w = w;
   p.valid_len = vl;
   p.out = out;
@@ -415,6 +433,8 @@ static int launch_score(const void* q, const void* kc, const float* w, int B, in
   p.tiles_per_cta = (int)tpc;
   p.ctas_per_group = cpg;
   p.key_per_row = per_row ? 1 : 0;
+  p.wait_ns = wait_limit();
+  p.fault = take_planted_fault();
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)(groups * cpg), 1, 1);
@@ -554,6 +574,8 @@ static int launch_score_hist(const void* q, const void* kc, const float* w, int 
   p.ctas_per_group = cpg;
   p.key_per_row = per_row ? 1 : 0;
   p.ghist = ghist;
+  p.wait_ns = wait_limit();
+  p.fault = take_planted_fault();
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)(((B + NT - 1) / NT) * cpg), 1, 1);
@@ -586,6 +608,7 @@ static int launch_hist_select(const float* scores, uint32_t* ghist, const int32_
   h.k = k;
   h.slice = ((S + C - 1) / C + 3) / 4 * 4;
   h.sorted = sorted;
+  h.status = s->status;
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)(B * C), 1, 1);
@@ -708,6 +731,8 @@ static int attention_enqueue(const uint16_t* q, const uint16_t* kv, long long kv
   for (int b0 = 0; b0 < B; b0 += per) {
     const int nb = std::min(per, B - b0);
     AttnParams p;
+    memset(&p, 0, sizeof(p));
+    p.wait_ns = wait_limit();
     p.kv = kv + (size_t)b0 * (size_t)kv_bstride_rows * D;
     p.kv_bstride = kv_bstride_rows * (long long)D;
     p.win = win ? win + (size_t)b0 * W * D : nullptr;
@@ -803,6 +828,8 @@ static int qproj_tc_enqueue(const void* x, const void* wq, const void* ww, int T
   if (!encode_rowblocks(ww ? ww : wq, ww ? heads : nq, d_in, 128, bpb, &tww)) return DS_ERR_ARG;
   if (!encode_rowblocks(x, T, d_in, kQtTok, bpb, &tx)) return DS_ERR_ARG;
   QtParams p;
+  memset(&p, 0, sizeof(p));
+  p.wait_ns = wait_limit();
   p.q = static_cast<uint16_t*>(q_out);
   p.w = w_out;
   p.status = s->status;
@@ -863,6 +890,20 @@ extern "C" int ds_get_device_status(void* stream) {
   return host;
 }
 
+extern "C" int ds_set_wait_limit(int64_t ns) {
+  if (ns < 0 || ns > kMaxWaitLimitNs) return DS_ERR_ARG;
+  g_wait_ns.store((long long)ns, std::memory_order_relaxed);
+  return DS_OK;
+}
+
+extern "C" int ds_plant_wait_fault(int launches) {
+  if (launches < 0) return DS_ERR_ARG;
+  g_planted.store(launches, std::memory_order_relaxed);
+  return DS_OK;
+}
+
+extern "C" int ds_debug_build(void) { return kDebugChecks ? 1 : 0; }
+
 extern "C" const char* ds_strerror(int code) {
   switch (code) {
     case DS_OK: return "DS_OK";
@@ -871,6 +912,7 @@ extern "C" const char* ds_strerror(int code) {
     case DS_ERR_TIMEOUT: return "DS_ERR_TIMEOUT: a bounded device wait ran out";
     case DS_ERR_UNSUPPORTED: return "DS_ERR_UNSUPPORTED: device is not sm_100";
     case DS_ERR_NOMEM: return "DS_ERR_NOMEM: scratch allocation failed";
+    case DS_ERR_RANGE: return "DS_ERR_RANGE: an input read on the device was out of range (DS_DEBUG build)";
     default: return "unknown status";
   }
 }
@@ -970,8 +1012,9 @@ extern "C" int ds_indexer_topk_noalloc(const void* q, const void* kcache, const 
   if (rc != DS_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // The scorer writes every position of every row (-inf at and past
-  // valid_len) before the selection reads it, so nothing left over from an
-  // earlier call is ever read and the array needs no clearing.
+  // valid_len, and -inf at the positions left when one of its waits runs
+  // out) before the selection reads it, so nothing left over from an earlier
+  // call is ever read and the array needs no clearing.
   rc = score_enqueue(q, kcache, w, batch, heads, S, valid_len, scores, st, s);
   if (rc != DS_OK) return rc;
   return topk_enqueue(scores, batch, S, k, DS_F32, valid_len, out_idx, out_score, out_score != nullptr, 0, st, s);

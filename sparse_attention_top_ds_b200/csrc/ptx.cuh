@@ -12,9 +12,11 @@ namespace dstopk {
 constexpr int kErrCuda = -2;     // DS_ERR_CUDA: a launch found its set-up inconsistent
 constexpr int kErrTimeout = -3;  // DS_ERR_TIMEOUT
 constexpr int kErrInternal = kErrCuda;
+constexpr int kErrRange = -6;    // DS_ERR_RANGE (recorded by DS_DEBUG builds only)
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s, unless the library is given another
+constexpr long long kMaxWaitLimitNs = 60000000000ll;  // the largest limit it may be given: 60 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -28,6 +30,22 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
+}
+
+// Bounds checks of the DS_DEBUG build.  An input the device reads that lies
+// outside its documented range (a valid length outside [0, n], an index past
+// the cache) is recorded as kErrRange in the status word; the kernel carries
+// on with the clamped value or skips the entry, as the release build does
+// without a word.  Nothing traps.
+#ifdef DS_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ void debug_range(bool in_range, int* status) {
+  if constexpr (kDebugChecks) {
+    if (!in_range) record_status(status, kErrRange);
+  }
 }
 
 // ------------------------------------------------------------------ mbarrier
@@ -65,15 +83,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of an mbarrier.  Gives up after kWaitLimitNs,
-// records kErrTimeout in *status and returns false; the caller carries on so
-// that every barrier the block or cluster still has to pass is still reached.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int* status) {
+// Wait for phase `parity` of an mbarrier.  Gives up after limit_ns (0: the
+// default kWaitLimitNs), records kErrTimeout in *status and returns false; the
+// caller carries on so that every barrier the block or cluster still has to
+// pass is still reached.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int* status,
+                                                  uint64_t limit_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
+  if (limit_ns == 0) limit_ns = kWaitLimitNs;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((it & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) {
       record_status(status, kErrTimeout);
       return false;
     }

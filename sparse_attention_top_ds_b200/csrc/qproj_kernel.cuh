@@ -188,6 +188,7 @@ struct QtParams {
   uint16_t* q;     // bf16 [T, nq]
   float* w;        // f32 [T, heads] or null
   int* status;
+  uint64_t wait_ns;        // limit of every bounded wait (0: the library default)
   int T, nq, heads, nblk;  // nblk = input width / 64
   int bpb;                 // 64-channel blocks per box (1 or 4)
   int nqb;                 // row blocks of Wq (nq / 128)
@@ -248,7 +249,7 @@ __global__ void __launch_bounds__(128, 1)
     bool ok = true;
     for (int i = 0; i < nbox && ok; ++i) {
       const int s = i % kQtStages;
-      ok = mbar_wait_bounded(full0 + 8u * s, (uint32_t)((i / kQtStages) & 1), p.status);
+      ok = mbar_wait_bounded(full0 + 8u * s, (uint32_t)((i / kQtStages) & 1), p.status, p.wait_ns);
       tc_fence_after();
       const uint32_t st = sbase + (uint32_t)s * kQtStage;
       const uint64_t a0 = sw128_kmajor_desc(st), x0 = sw128_kmajor_desc(st + kQtWBox);
@@ -260,7 +261,7 @@ __global__ void __launch_bounds__(128, 1)
       }
       mma_commit(empty0 + 8u * s);
       if (ok && i + kQtStages < nbox) {
-        ok = mbar_wait_bounded(empty0 + 8u * s, (uint32_t)((i / kQtStages) & 1), p.status);
+        ok = mbar_wait_bounded(empty0 + 8u * s, (uint32_t)((i / kQtStages) & 1), p.status, p.wait_ns);
         if (ok) load(i + kQtStages);  // refill only a stage its MMAs have finished with
       }
     }
@@ -268,7 +269,7 @@ __global__ void __launch_bounds__(128, 1)
   }
 
   // ---- epilogue: thread = weight row (TMEM lane), 16 token columns
-  mbar_wait_bounded(bar_done, 0, p.status);
+  mbar_wait_bounded(bar_done, 0, p.status, p.wait_ns);
   __syncwarp();
   tc_fence_after();
   uint32_t r[16];
@@ -290,7 +291,7 @@ __global__ void __launch_bounds__(128, 1)
                      : "memory");
     } else {
       if ((row & 63) == 0) mbar_arrive_expect_tx(bar_recv, 64 * kQtTok * 4);
-      mbar_wait_bounded(bar_recv, 0, p.status);
+      mbar_wait_bounded(bar_recv, 0, p.status, p.wait_ns);
 #pragma unroll
       for (int t = 0; t < kQtTok; ++t)
         r[t] = __float_as_uint(__uint_as_float(r[t]) + recv[(row & 63) * kQtTok + t]);

@@ -253,6 +253,7 @@ struct HsParams {
   int B, S, k;
   int slice;                // positions per CTA, a multiple of 4
   int sorted;
+  int* status;              // device status word (DS_DEBUG range checks)
 };
 
 // Shared memory of topk_hist_select_kernel (about 23 KiB, so that several CTAs
@@ -300,6 +301,7 @@ __global__ void __launch_bounds__(kHsThreads) topk_hist_select_kernel(const HsPa
   int L = p.S;
   if (p.valid_len) {
     const int v = p.valid_len[row];
+    if (tid == 0 && crank == 0) debug_range(v >= 0 && v <= p.S, p.status);
     L = v < 0 ? 0 : (v > p.S ? p.S : v);
   }
   const int kk = min(p.k, L);
@@ -472,13 +474,14 @@ __global__ void __launch_bounds__(kHsThreads) topk_hist_select_kernel(const HsPa
   uint32_t* sv = cand_raw;
   for (int j = tid; j < kk; j += kHsThreads) {
     const uint32_t pos = (uint32_t)__ldcg(out_idx + j);
-    sp[j] = pos;
-    sv[j] = __ldcg(srow + pos);
+    const bool in = pos < (uint32_t)L;  // always, unless the row's histogram disagreed with its scores
+    sp[j] = in ? pos : 0xFFFFFFFFu;
+    sv[j] = in ? __ldcg(srow + pos) : 0u;
   }
   __syncthreads();
   mr_sort_pairs<kHsThreads>(sp, sv, 1, [&](int) { return (uint32_t)kk; });
   for (int j = tid; j < kk; j += kHsThreads) {
-    out_idx[j] = (int32_t)sp[j];
+    out_idx[j] = sp[j] == 0xFFFFFFFFu ? -1 : (int32_t)sp[j];
     if (out_score) out_score[j] = __uint_as_float(sv[j]);
   }
 }

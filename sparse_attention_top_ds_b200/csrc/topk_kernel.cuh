@@ -292,6 +292,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) topk_cluster_kernel(const TopkP
   int L = p.n;
   if (p.valid_len) {
     const int v = p.valid_len[row];
+    if (tid == 0 && crank == 0) debug_range(v >= 0 && v <= p.n, p.status);
     L = v < 0 ? 0 : (v > p.n ? p.n : v);
   }
   const int kk = min(p.k, L);

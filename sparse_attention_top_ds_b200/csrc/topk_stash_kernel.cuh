@@ -56,6 +56,7 @@ struct TsParams {
   int slice;         // elements per CTA, a multiple of 8
   int return_value;
   int sorted;
+  int* status;       // device status word (DS_DEBUG range checks)
 };
 
 struct TsCtrl {
@@ -343,6 +344,7 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   int L = p.n;
   if (p.valid_len) {
     const int v = p.valid_len[row];
+    if (tid == 0 && crank == 0) debug_range(v >= 0 && v <= p.n, p.status);
     L = v < 0 ? 0 : (v > p.n ? p.n : v);
   }
   const int kk = min(p.k, L);

@@ -46,11 +46,53 @@ def test_exported_symbols_have_c_linkage(lib):
     assert set(declared_entry_points()) <= exported
 
 
+@pytest.fixture(scope="module")
+def debug_lib(lib):
+    from sparse_attention_top_ds_b200 import build
+    assert os.path.exists(build.LIB_DEBUG), "build() makes libdstopk_debug.so beside libdstopk.so"
+    return ctypes.CDLL(build.LIB_DEBUG)
+
+
+def test_debug_build_flag_plumbing(lib, debug_lib):
+    # the DS_DEBUG compile flag reaches the device code's range checks: the
+    # release library reports 0, the debug library 1, and both export the
+    # same boundary with C linkage
+    from sparse_attention_top_ds_b200 import build
+    assert lib.ds_debug_build() == 0
+    assert debug_lib.ds_debug_build() == 1
+    for name in declared_entry_points():
+        assert hasattr(debug_lib, name), f"{name} is not exported by the debug build"
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB_DEBUG], capture_output=True, text=True).stdout
+    assert set(declared_entry_points()) <= set(re.findall(r"\bT (ds_\w+)$", out, flags=re.M))
+    debug_lib.ds_strerror.restype = ctypes.c_char_p
+    assert b"DS_ERR_RANGE" in debug_lib.ds_strerror(-6)
+
+
+def test_debug_build_is_rebuilt_with_the_release_build():
+    # the build compiles the debug library with -DDS_DEBUG and the release one without
+    from sparse_attention_top_ds_b200 import build
+    src = open(build.__file__).read()
+    assert '"-DDS_DEBUG"' in src
+    assert not build.stale(build.LIB) and not build.stale(build.LIB_DEBUG)
+
+
+def test_wait_limit_and_planted_fault_arguments_need_no_gpu(lib):
+    lib.ds_set_wait_limit.argtypes = [ctypes.c_int64]
+    lib.ds_plant_wait_fault.argtypes = [ctypes.c_int]
+    assert lib.ds_set_wait_limit(-1) == -1
+    assert lib.ds_set_wait_limit(60_000_000_001) == -1
+    assert lib.ds_set_wait_limit(1_000_000) == 0
+    assert lib.ds_set_wait_limit(0) == 0
+    assert lib.ds_plant_wait_fault(-1) == -1
+    assert lib.ds_plant_wait_fault(0) == 0
+
+
 def test_strerror(lib):
     lib.ds_strerror.restype = ctypes.c_char_p
     assert lib.ds_strerror(0) == b"DS_OK"
     assert b"argument" in lib.ds_strerror(-1)
     assert b"unknown" in lib.ds_strerror(12345)
+    assert b"DS_ERR_RANGE" in lib.ds_strerror(-6)
 
 
 def test_argument_errors_need_no_gpu(lib):
