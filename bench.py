@@ -378,9 +378,20 @@ def measure_compress(ds, inputs, dev, rank):
             "bytes_per_call": int(rows.nbytes + gate.nbytes + 8 * 512 * 2)}
 
 
-def run_attention_only(args):
-    """`--only attention` / `--only qproj`: one beside-the-headline measurement
-    alone (the commands the profiles of those kernels are taken with)."""
+ONLY_WORKLOADS = {
+    "decode": "decode indexer + top-k: 8 rows x 64 heads x 128 bf16 vs 32768 keys, valid_len ~ U{4096..32768}, "
+              "k = 1024, scores returned",
+    "sampling": "top-k of 64 x 129280 float32 sampling rows, k = 1024, values and indices",
+    "indexer-rows": "top-k of 64 x 131072 bfloat16 indexer-style rows, k = 2048, indices only",
+    "prefill": "prefill indexer + top-k: 4096 rows x 64 heads x 128 bf16 vs 32768 keys, causal valid_len, k = 2048",
+}
+
+
+def run_only(args):
+    """`--only <part>`: one part of the step alone, for profiling (the commands
+    the profiles are taken with): the sparse attention, the query projection,
+    or one workload of the selection step timed over `steps` plain calls
+    (one input, so the times of inputs smaller than L2 are L2-warm)."""
     import torch
     import sparse_attention_top_ds_b200 as ds
     from sparse_attention_top_ds_b200 import inputs
@@ -391,9 +402,46 @@ def run_attention_only(args):
     stream = torch.cuda.current_stream()
     if args.only == "qproj":
         key, a = "qproj", measure_qproj(ds, inputs, dev, stream, rank, hbm_gbs, args.steps, warmup=args.warmup)
-    else:
+    elif args.only == "attention":
         key, a = "sparse_attention", measure_attention(ds, inputs, dev, stream, rank, hbm_gbs, tflops, args.steps,
                                                        warmup=args.warmup)
+    else:
+        to = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+        if args.only in ("decode", "prefill"):
+            if args.only == "decode":
+                q, kc, w, vl = inputs.decode(seed=inputs.SEED_DECODE + rank)
+                k = DECODE["k"]
+            else:
+                q, kc, w, vl = inputs.prefill(seed=inputs.SEED_PREFILL + rank)
+                k = PREFILL["k"]
+            qd, kd, wd, vd = to(q), to(kc), torch.from_numpy(w).to(dev), torch.from_numpy(vl).to(dev)
+            oi = torch.empty((q.shape[0], k), dtype=torch.int32, device=dev)
+            osc = torch.empty((q.shape[0], k), dtype=torch.float32, device=dev)
+            fn = lambda: ds.ds_indexer_topk(qd, kd, wd, k, valid_len=vd, return_score=True, out_idx=oi, out_score=osc)
+        elif args.only == "sampling":
+            x = torch.from_numpy(inputs.sampling(seed=inputs.SEED_SAMPLING + rank)[0]).to(dev)
+            oi = torch.empty((x.shape[0], 1024), dtype=torch.int32, device=dev)
+            ov = torch.empty((x.shape[0], 1024), dtype=torch.float32, device=dev)
+            fn = lambda: ds.ds_topk(x, 1024, return_value=True, out_idx=oi, out_val=ov)
+        else:  # indexer-rows
+            q, kc, w = inputs.indexer_factors(seed=inputs.SEED_INDEXER + rank, batch=64, n=131072)
+            x = ds.ds_indexer_score(to(q), to(kc), torch.from_numpy(w).to(dev)).to(torch.bfloat16)
+            oi = torch.empty((64, 2048), dtype=torch.int32, device=dev)
+            fn = lambda: ds.ds_topk(x, 2048, return_value=False, out_idx=oi)
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a0, b0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b0.record(stream)
+        torch.cuda.synchronize()
+        status = ds.ds_get_device_status()
+        if status != ds.DS_OK:
+            raise RuntimeError(f"device status: {ds.strerror(status)}")
+        key, a = args.only, {"workload": ONLY_WORKLOADS[args.only],
+                             "us_per_call": round(a0.elapsed_time(b0) * 1e3 / max(1, args.steps), 2)}
     if rank == 0:
         print(json.dumps({key: a, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup}), flush=True)
 
@@ -716,8 +764,6 @@ def run_ours(args):
     e2e_dec_h2d = q_pin.numel() * 2 + w_pin.numel() * 4 + vl_pin.numel() * 4
     e2e_dec_d2h = didx_pin.numel() * 4
 
-    # DRAM bytes per launch of the dominant kernel from one ncu capture; null
-    # once the kernel's source has changed since that capture
     # ---- prefill, reported beside the headline: 4096 query rows x 64 heads
     # against 32768 keys, causal valid_len, k = 2048 (indexer + top-k per call,
     # and the scorer alone for its tensor-pipe fraction)
@@ -763,6 +809,8 @@ def run_ours(args):
     qproj = measure_qproj(ds, inputs, dev, stream, rank, hbm_gbs, ATTN_CALLS)
     compress = measure_compress(ds, inputs, dev, rank)
 
+    # DRAM bytes per launch of the dominant kernel from one ncu capture; null
+    # once the kernel's source has changed since that capture
     traffic = None
     prof = os.path.join(ROOT, "profiles", "topk_traffic.json")
     try:
@@ -850,15 +898,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "attention", "qproj"], default="all",
-                    help="time the sparse attention or the query projection alone (profiling)")
+    ap.add_argument("--only", choices=["all", "attention", "qproj"] + list(ONLY_WORKLOADS), default="all",
+                    help="time one part of the step alone (profiling): the sparse attention, the query "
+                         "projection, or one selection workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
-    elif args.only in ("attention", "qproj"):
-        run_attention_only(args)
+    elif args.only != "all":
+        run_only(args)
     else:
         run_ours(args)
     import torch.distributed as dist

@@ -6,11 +6,22 @@ framework's allocation-free graph capture, latency-bound paths): its score rows
 live in a fixed array inside the library.  Its results must match the regular
 ds_indexer_topk, which uses the library's grow-only scratch buffer, within the
 tolerance the indexer tests use, on two calls in a row with different inputs
-(the fixed array keeps the previous call's contents).  This file runs last so
-that a stop-at-first-failure run has already run every other test.
+(the fixed array keeps the previous call's contents), and the oracle's
+selection.  Two child processes show that the first call allocates nothing:
+with every module loaded up front and the library's device set-up done, the
+device's free memory is the same before and after it (while a first regular
+call takes its scratch); and a first call captured into a CUDA graph -- where
+a cudaMalloc would end the capture with an error -- replays correctly, at
+batch * S past anything the regular scratch holds at that point.  This file
+runs last so that a stop-at-first-failure run has already run every other
+test.
 """
 
 import ctypes
+import json
+import os
+import subprocess
+import sys
 
 import numpy as np
 import pytest
@@ -18,6 +29,8 @@ import torch
 
 import sparse_attention_top_ds_b200 as ds
 from sparse_attention_top_ds_b200 import _native, inputs
+
+from test_indexer_gpu import check_selection
 
 pytestmark = pytest.mark.gpu
 
@@ -86,3 +99,97 @@ def test_noalloc_rejects_sizes_beyond_the_fixed_array(cuda_device):
                                      ctypes.c_void_p(wd.data_ptr()), B, 64, 128, S, None, 16,
                                      ctypes.c_void_p(idx.data_ptr()), None, stream)
     assert rc == ds.DS_ERR_ARG
+
+
+def test_noalloc_matches_the_oracle(cuda_device):
+    lib = _native.load()
+    for seed, B, S, k, vl in ((91, 8, 32768, 1024, None), (92, 6, 9000, 2048, [9000, 0, 1, 8999, 4500, -2]),
+                              (93, 64, 4096, 512, None)):
+        q, kc, w = inputs.indexer_factors(seed=seed, batch=B, n=S)
+        vln = None if vl is None else np.array(vl, dtype=np.int32)
+        args = (_dev_bf16(q), _dev_bf16(kc), torch.from_numpy(w).cuda(),
+                None if vln is None else torch.from_numpy(vln).cuda())
+        idx, score = _call(lib.ds_indexer_topk_noalloc, *args, k)
+        check_selection(q, kc, w, vln, k, idx, score)
+
+
+_CHILD_MEMINFO = r"""
+import json, sys
+import numpy as np
+import torch
+sys.path.insert(0, sys.argv[1])
+import sparse_attention_top_ds_b200 as ds
+from sparse_attention_top_ds_b200 import inputs
+torch.cuda.set_device(0)
+q, kc, w, vl = inputs.decode()
+bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+qd, kd, wd, vd = bf(q), bf(kc), torch.from_numpy(w).cuda(), torch.from_numpy(vl).cuda()
+idx = torch.empty((8, 1024), dtype=torch.int32, device="cuda")
+sc = torch.empty((8, 1024), dtype=torch.float32, device="cuda")
+# the library's one-time device set-up (kernel attributes, the status word's
+# address); the CUDA driver reserves a few MiB of its own on that first use
+ds.ds_get_device_status()
+torch.cuda.synchronize()
+free0 = torch.cuda.mem_get_info()[0]
+ds.ds_indexer_topk_noalloc(qd, kd, wd, 1024, valid_len=vd, return_score=True, out_idx=idx, out_score=sc)
+torch.cuda.synchronize()
+free1 = torch.cuda.mem_get_info()[0]
+status = ds.ds_get_device_status()
+ds.ds_indexer_topk(qd, kd, wd, 1024, valid_len=vd, out_idx=idx)
+torch.cuda.synchronize()
+free2 = torch.cuda.mem_get_info()[0]
+print("RESULT " + json.dumps({"free0": free0, "free1": free1, "free2": free2, "status": status}))
+"""
+
+_CHILD_CAPTURE = r"""
+import json, sys
+import numpy as np
+import torch
+sys.path.insert(0, sys.argv[1]); sys.path.insert(0, sys.argv[1] + "/tests")
+import sparse_attention_top_ds_b200 as ds
+from sparse_attention_top_ds_b200 import inputs
+from test_indexer_gpu import check_selection
+torch.cuda.set_device(0)
+bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+# a small regular call first: the library's own scratch now holds 2 x 1000 scores
+qs, ks, ws = inputs.indexer_factors(seed=3, batch=2, n=1000)
+ds.ds_indexer_topk(bf(qs), bf(ks), torch.from_numpy(ws).cuda(), 10)
+torch.cuda.synchronize()
+# then the first allocation-free call, 8 x 32768 positions, inside a graph capture
+q, kc, w, vl = inputs.decode(seed=5)
+qd, kd, wd, vd = bf(q), bf(kc), torch.from_numpy(w).cuda(), torch.from_numpy(vl).cuda()
+idx = torch.full((8, 1024), -7, dtype=torch.int32, device="cuda")
+sc = torch.empty((8, 1024), dtype=torch.float32, device="cuda")
+g = torch.cuda.CUDAGraph()
+with torch.cuda.graph(g, capture_error_mode="thread_local"):
+    ds.ds_indexer_topk_noalloc(qd, kd, wd, 1024, valid_len=vd, return_score=True, out_idx=idx, out_score=sc,
+                               stream=torch.cuda.current_stream())
+g.replay()
+torch.cuda.synchronize()
+status = ds.ds_get_device_status()
+check_selection(q, kc, w, vl, 1024, idx.cpu().numpy(), sc.cpu().numpy())
+print("RESULT " + json.dumps({"status": status}))
+"""
+
+
+def _child(code, extra_env=None):
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ)
+    env.update(extra_env or {})
+    out = subprocess.run([sys.executable, "-c", code, root], env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stdout[-2000:] + out.stderr[-4000:]
+    line = [ln for ln in out.stdout.splitlines() if ln.startswith("RESULT ")][-1]
+    return json.loads(line[len("RESULT "):])
+
+
+def test_first_noalloc_call_leaves_free_memory_unchanged(cuda_device):
+    r = _child(_CHILD_MEMINFO, {"CUDA_MODULE_LOADING": "EAGER"})
+    assert r["status"] == ds.DS_OK
+    assert r["free1"] == r["free0"], f"the first allocation-free call took {r['free0'] - r['free1']} bytes"
+    # the control: the regular entry point's first call does allocate its scratch
+    assert r["free2"] < r["free1"]
+
+
+def test_first_noalloc_call_captures_into_a_graph(cuda_device):
+    r = _child(_CHILD_CAPTURE)
+    assert r["status"] == ds.DS_OK
