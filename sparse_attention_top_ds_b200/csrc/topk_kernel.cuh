@@ -66,6 +66,17 @@ struct F32Keys {
   __device__ __forceinline__ static uint32_t slot(const uint4& v, int j) {
     return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
   }
+  // The smallest value whose key is >= t, as a float: key(x) >= t holds
+  // exactly when !(x < bound(t)) for every x that is not a NaN, and a NaN x
+  // passes too (it has the top key).  For t above key(+inf), and t below
+  // key(-inf), bound(t) is a NaN and every x passes: a superset, never a miss.
+  __device__ __forceinline__ static float bound(uint32_t t) {
+    return __uint_as_float((t & 0x80000000u) ? (t & 0x7FFFFFFFu) : ~t);
+  }
+  // !(element j of v < tf): one float compare instead of a key conversion
+  __device__ __forceinline__ static bool ge(const uint4& v, int j, float tf) {
+    return !(__uint_as_float(slot(v, j)) < tf);
+  }
 };
 
 // bfloat16 rows: 16-bit keys; digits 12 (pass 0), then 4.
@@ -85,6 +96,14 @@ struct BF16Keys {
   __device__ __forceinline__ static uint32_t slot(const uint4& v, int j) {
     const uint32_t w = (j >> 1) == 0 ? v.x : ((j >> 1) == 1 ? v.y : ((j >> 1) == 2 ? v.z : v.w));
     return (j & 1) ? (w >> 16) : (w & 0xFFFFu);
+  }
+  // as F32Keys::bound, for 16-bit keys (a bfloat16 is the top half of a float)
+  __device__ __forceinline__ static float bound(uint32_t t) {
+    return __uint_as_float(((t & 0x8000u) ? (t & 0x7FFFu) : (~t & 0xFFFFu)) << 16);
+  }
+  __device__ __forceinline__ static bool ge(const uint4& v, int j, float tf) {
+    const uint32_t w = (j >> 1) == 0 ? v.x : ((j >> 1) == 1 ? v.y : ((j >> 1) == 2 ? v.z : v.w));
+    return !(__uint_as_float((j & 1) ? (w & 0xFFFF0000u) : (w << 16)) < tf);
   }
 };
 

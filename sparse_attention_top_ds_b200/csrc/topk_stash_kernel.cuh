@@ -17,10 +17,16 @@
 //    k largest, so a CTA only checks its own count: the stash must hold at
 //    least min(k, slice) keys and fit.  In a cluster every CTA then copies its
 //    stash into the leader CTA (distributed shared memory).
-//  * The leader selects the k largest of the stash by (key, lower position):
-//    one radix pass over the stash per digit (and, for keys equal to the k-th,
-//    over positions);
-//    every selected entry is written out with one warp-level atomic per
+//  * While it stashes, each CTA counts the stashed keys in a histogram of
+//    their offset above t (4096 bins of 2^12 float32 keys, or of single
+//    bfloat16 keys; the last bin takes everything above).  The leader adds
+//    the CTAs' histograms, finds the bin of the row's k-th key in it, and
+//    resolves only that bin: one radix pass over the stash's keys inside it
+//    (none for bfloat16), then positions for ties.  When the k-th key lies in
+//    the last bin (or a CTA's stash was redone, see below), the leader instead
+//    selects from the whole stash, one radix pass per digit below the
+//    common prefix of its smallest and largest key.
+//    Every selected entry is written out with one warp-level atomic per
 //    visit, and sorted_index sorts the selection by position first.
 //  * A CTA whose stash came out short or too long (an unlucky sample, many
 //    equal keys) re-reads its slice from L2 and finds its exact k-th (key,
@@ -69,10 +75,12 @@ struct TsCtrl {
   uint32_t wex[33];         // scan scratch: their exclusive prefixes, then the total
   uint32_t part[32][kTsMaxCluster];  // per-warp partial counts
   uint32_t above_of[kTsMaxCluster];
+  uint32_t tval[16];        // every CTA: each CTA's stash threshold
 };
 
-// Shared memory, in order: radix histogram u32[4096] (later the sorted
-// selection: positions u32[2048], raw scores u32[2048]) | control | this CTA's
+// Shared memory, in order: histogram u32[4096] (the stash's offsets above the
+// threshold during the stream, then the radix passes' histogram, then the
+// sorted selection: positions u32[2048], raw scores u32[2048]) | control | this CTA's
 // stash (raw u32[cap], position u32[cap]) | cp.async ring of kTsStages stages.
 // The last ring stage holds the sample's histogram until the ring reaches it.
 // In a cluster the leader receives the stash of CTA c >= 1 in its ring (free
@@ -271,6 +279,19 @@ __device__ __forceinline__ void ts_block_minmax(uint32_t lo, uint32_t hi, TsCtrl
   gmax = ctrl->bcast[1];
 }
 
+// One slot of *counter to each lane of a warp that asks (all 32 lanes call
+// it): a ballot, one atomic, a population count.
+__device__ __forceinline__ uint32_t ts_warp_alloc1(bool take, uint32_t* counter) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
+  uint32_t base = 0u;
+  if (m != 0u) {
+    if (lane == 0) base = atomicAdd(counter, (uint32_t)__popc(m));
+    base = __shfl_sync(0xFFFFFFFFu, base, 0);
+  }
+  return base + (uint32_t)__popc(m & ((1u << lane) - 1u));
+}
+
 // Hands out n consecutive slots of *counter to each lane of a warp (all 32
 // lanes call it); returns this lane's first slot.
 __device__ __forceinline__ uint32_t ts_warp_alloc(uint32_t n, uint32_t* counter) {
@@ -383,6 +404,10 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
     ctrl->cnt = 0u;
     ctrl->out = 0u;
   }
+  // the histogram of the stashed keys' offsets above t, counted after the
+  // stream (zeroed before the first barrier below)
+  constexpr int kRel = K::kBits == 32 ? 12 : 0;
+  for (int i = tid; i < 4096; i += NT) hist[i] = 0u;
 
   // ---- a strided sample of the full words (64 evenly spaced runs of run_w
   // words) when the slice does not fit the stash whole
@@ -439,6 +464,9 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
     const uint32_t b0 = ts_find_bin<NT>(shist, 4096, (uint32_t)kk, ctrl, above, inbin);
     t = b0 << kShift0;
   } else if (sampled) {
+    // the stream's first stages load while the sample is counted (the
+    // histogram lives in the ring's last stage, loaded later)
+    for (int st = 0; st < kTsStages - 1; ++st) issue(st);
     for (int i = tid; i < 4096; i += NT) shist[i] = 0u;
     __syncthreads();
 #pragma unroll
@@ -448,7 +476,6 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
         for (int e = 0; e < K::kVec; ++e) atomicAdd(shist + (K::key(K::slot(s[j], e)) >> kShift0), 1u);
       }
     }
-    for (int st = 0; st < kTsStages - 1; ++st) issue(st);  // the sample has landed: start the stream
     __syncthreads();
     const int ns = sw * K::kVec;
     const float lam = (float)need * (float)ns / (float)m;
@@ -482,14 +509,17 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
     __syncthreads();  // the zeroed histogram and counters
   }
 
-  // ---- one pass: every key >= t is stashed with its position and its first
-  // digit counted; a warp takes its stash slots with one atomic per stage
+  // ---- one pass: every key >= t is stashed with its position; a warp takes
+  // its stash slots with one atomic per stage.  The test is a float compare
+  // against bound(t) (exact, or a superset that the stash's checks catch); the
+  // per-element hit mask is built only by threads with a hit.
+  const float tf = K::bound(t);
   for (int st = 0; st < nst; ++st) {
     issue(st + kTsStages - 1);
     asm volatile("cp.async.wait_group %0;" ::"n"(kTsStages - 1) : "memory");
     const int slot = st % kTsStages;
     uint4 x[V];
-    unsigned long long hits = 0ull;
+    bool anyh = false;
 #pragma unroll
     for (int v = 0; v < V; ++v) {
       const int w = st * stage_words + v * NT + tid;
@@ -497,8 +527,18 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
       if (w < nfull) {
         x[v] = *reinterpret_cast<const uint4*>(ring + ((size_t)slot * stage_words + v * NT + tid) * 16);
 #pragma unroll
-        for (int j = 0; j < K::kVec; ++j)
-          hits |= (unsigned long long)(K::key(K::slot(x[v], j)) >= t) << (v * K::kVec + j);
+        for (int j = 0; j < K::kVec; ++j) anyh |= K::ge(x[v], j, tf);
+      }
+    }
+    unsigned long long hits = 0ull;
+    if (anyh) {
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        if (st * stage_words + v * NT + tid < nfull) {
+#pragma unroll
+          for (int j = 0; j < K::kVec; ++j)
+            hits |= (unsigned long long)K::ge(x[v], j, tf) << (v * K::kVec + j);
+        }
       }
     }
     uint32_t pos = ts_warp_alloc((uint32_t)__popcll(hits), &ctrl->cnt);
@@ -532,6 +572,17 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   }
   __syncthreads();
 
+  // the offset histogram of the stash's keys >= t (a complete stash only)
+  {
+    const uint32_t n = ctrl->cnt;
+    if (n <= (uint32_t)kTsCap) {
+      for (int i = tid; i < (int)n; i += NT) {
+        const uint32_t key = K::key(st_raw[i]);
+        if (key >= t) atomicAdd(hist + min(4095u, (key - t) >> kRel), 1u);
+      }
+    }
+  }
+
   // ---- in a cluster, every stash and histogram goes to the leader: stash c
   // into the leader's ring (free once every CTA has streamed) at (c - 1) stash
   // sizes, histogram c into its slot c
@@ -555,8 +606,34 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   uint32_t cnt = ctrl->cnt;
   const bool ok = (counted || cnt >= (uint32_t)need) && cnt <= (uint32_t)kTsCap;
   bool all_ok = ok;
+  // The offset histograms meet in one frame: tmax, the largest of the CTAs'
+  // thresholds.  With every stash complete, the row's k-th key is >= each
+  // threshold of a slice that holds k keys (and slices that hold fewer have
+  // t = 0), so every key at or above the k-th is >= tmax and in a stash.
+  // CTA c's bin i is bin i - dc of that frame (dc = (tmax - t_c) >> kRel);
+  // its bins below dc drop out and its last bin stays the last.
+  uint32_t tmax = t, dmax = 0u;
+  uint32_t* acc = hist;  // the leader's merged histogram
   if (C > 1) {
+    acc = shist;  // the ring's last stage: free after the stream, clear of the received stashes
+    if (crank == 0)
+      for (int i = tid; i < 4096; i += NT) acc[i] = 0u;
+    if (tid < C) dsmem_st_u32(dsmem_map(smem_u32(&ctrl->tval[crank]), (uint32_t)tid), t);
     cluster_sync();  // every CTA has streamed: the leader's ring is free
+    for (int c = 0; c < C; ++c) tmax = max(tmax, ctrl->tval[c]);
+    for (int c = 0; c < C; ++c) dmax = max(dmax, (tmax - ctrl->tval[c]) >> kRel);
+    if (ok) {
+      const uint32_t dc = (tmax - t) >> kRel;
+      const uint32_t la = dsmem_map(smem_u32(acc), 0);
+      for (int i = tid; i < 4096; i += NT) {
+        const uint32_t h = hist[i];
+        if (h && (uint32_t)i >= dc) {
+          const uint32_t j = i == 4095 ? 4095u : (uint32_t)i - dc;
+          if (crank == 0) atomicAdd(acc + j, h);
+          else dsmem_red_add_u32(la + 4u * j, h);
+        }
+      }
+    }
     if (ok && crank != 0) ship(cnt);
     if (tid < C) dsmem_st_u32(dsmem_map(smem_u32(&ctrl->ok[crank]), (uint32_t)tid), ok ? 1u : 0u);
     cluster_sync();
@@ -630,19 +707,50 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
       if (i < nc) f(K::key(rr[i]), rp[i]);
     }
   };
-  // the stash's keys share their top bits between its smallest and largest
-  // key: the radix digits start below that common prefix, so the first pass
-  // spreads the stash over many bins
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  visit_stash([&](uint32_t key, uint32_t) {
-    lo = min(lo, key);
-    hi = max(hi, key);
-  });
-  uint32_t gmin, gmax;
-  ts_block_minmax<NT>(lo, hi, ctrl, gmin, gmax);
-  const int common = gmin == gmax ? K::kBits : __clz(gmin ^ gmax) - (32 - K::kBits);
-  const int shift0 = K::kBits - common;
-  const TsCut cut = ts_select<K, NT>(visit_stash, kk, hist, ctrl, ts_top(gmax, shift0), shift0);
+  // With every stash as streamed, the offset histogram counts exactly the
+  // stash's keys >= t: the bin fb of the k-th key, and only that bin to
+  // resolve (mode 1: all of it is taken; mode 2: a cut inside it).
+  int mode = 0;
+  uint32_t fb = 0u;
+  TsCut cut = TsCut{0u, 0, 0u};
+  if (all_ok) {
+    uint32_t above, inbin;
+    const uint32_t b = ts_find_bin<NT>(acc, 4096, (uint32_t)kk, ctrl, above, inbin);
+    // (bins 4095 - dc .. 4094 lack CTA c's keys counted in its last bin, so
+    // only a bin below all of them is exact)
+    if (b + dmax < 4095u && above < (uint32_t)kk && above + inbin >= (uint32_t)kk) {
+      fb = b;
+      const int krem = kk - (int)above;
+      if (inbin == (uint32_t)krem) {
+        mode = 1;
+      } else {
+        mode = 2;
+        cut = ts_select<K, NT>(visit_stash, krem, hist, ctrl, (tmax >> kRel) + b, kRel);
+      }
+    }
+  }
+  if (mode == 0) {
+    // the stash's keys share their top bits between its smallest and largest
+    // key: the radix digits start below that common prefix, so the first pass
+    // spreads the stash over many bins
+    __syncthreads();
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    visit_stash([&](uint32_t key, uint32_t) {
+      lo = min(lo, key);
+      hi = max(hi, key);
+    });
+    uint32_t gmin, gmax;
+    ts_block_minmax<NT>(lo, hi, ctrl, gmin, gmax);
+    const int common = gmin == gmax ? K::kBits : __clz(gmin ^ gmax) - (32 - K::kBits);
+    const int shift0 = K::kBits - common;
+    cut = ts_select<K, NT>(visit_stash, kk, hist, ctrl, ts_top(gmax, shift0), shift0);
+  }
+  auto taken = [&](uint32_t key, uint32_t pos) -> bool {
+    if (mode == 0) return ts_taken(cut, key, pos);
+    if (key < tmax) return false;
+    const uint32_t rel = min(4095u, (key - tmax) >> kRel);
+    return rel > fb || (rel == fb && (mode == 1 || ts_taken(cut, key, pos)));
+  };
   // every selected entry (exactly kk): one warp-level slot allocation per
   // visit; with sorted_index gathered in shared memory first
   uint32_t* sel_pos = hist;
@@ -659,9 +767,9 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
       if (i < nc) {
         raw = rr[i];
         pos = rp[i];
-        take = ts_taken(cut, K::key(raw), pos);
+        take = taken(K::key(raw), pos);
       }
-      const uint32_t slot = ts_warp_alloc(take ? 1u : 0u, &ctrl->out);
+      const uint32_t slot = ts_warp_alloc1(take, &ctrl->out);
       if (take && slot < (uint32_t)kk) {
         if (sorted) {
           sel_pos[slot] = pos;

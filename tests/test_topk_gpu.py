@@ -163,6 +163,35 @@ def test_signed_zeros_nan_and_infinities(cuda_device, dtype):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_thresholds_on_special_values(cuda_device, dtype):
+    # long rows (the stash kernel streams them) whose k-th key is a NaN (more
+    # NaNs of every payload and sign than k), a subnormal, a zero of either
+    # sign, or -inf
+    n = 40000
+    g = np.random.default_rng(9)
+    if dtype == "f32":
+        nans = np.array([0x7FC00000, 0xFFC00000, 0x7F800001, 0xFFFFFFFF], dtype=np.uint32)
+        sub = lambda m: g.integers(1, 0x007FFFFF, size=m, dtype=np.uint32)
+        pz, nz, ninf, sign = 0x00000000, 0x80000000, 0xFF800000, 0x80000000
+        raw = g.standard_normal((4, n), dtype=np.float32).view(np.uint32).copy()
+    else:
+        nans = np.array([0x7FC0, 0xFFC0, 0x7F81, 0xFFFF], dtype=np.uint16)
+        sub = lambda m: g.integers(1, 0x007F, size=m, dtype=np.uint16)
+        pz, nz, ninf, sign = 0x0000, 0x8000, 0xFF80, 0x8000
+        raw = inputs.f32_to_bf16_bits(g.standard_normal((4, n), dtype=np.float32)).copy()
+    raw[0, g.choice(n, 12000, replace=False)] = g.choice(nans, 12000)
+    raw[1] = sub(n) | np.where(g.random(n) < 0.5, sign, 0).astype(raw.dtype)
+    raw[1, g.choice(n, 3000, replace=False)] = pz
+    raw[1, g.choice(n, 3000, replace=False)] = nz
+    raw[2, :] = ninf
+    raw[2, g.choice(n, 500, replace=False)] = raw[3, :500]
+    raw[3, :] = np.where(g.random(n) < 0.5, pz, nz).astype(raw.dtype)
+    raw[3, g.choice(n, 300, replace=False)] = sub(300) | sign
+    for k in (100, 2048):
+        run_case(raw, dtype, k)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_ascending_and_descending(cuda_device, dtype):
     x = np.arange(100000, dtype=np.float32)[None, :].repeat(2, axis=0)
     x[1] = x[1][::-1]
