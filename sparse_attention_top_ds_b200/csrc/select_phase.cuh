@@ -265,9 +265,12 @@ struct HsSmem {
   static constexpr int kOffCand = kOffHist;
   static constexpr int kOffPass = kOffHist + kSelBins * 4;  // u32[1024]
   static constexpr int kOffCtrl = kOffPass + (1 << kSelDigit) * 4;  // MrCtrl, TsCtrl, RowSel
-  static constexpr int kBytes =
-      kOffCtrl + (int)((sizeof(MrCtrl<1, kHsThreads>) + sizeof(TsCtrl) + sizeof(RowSel) + 127) / 128 * 128);
+  // each control block on a 16-byte boundary (TsCtrl holds 8-byte mbarriers)
+  static constexpr int kOffTs = kOffCtrl + (int)((sizeof(MrCtrl<1, kHsThreads>) + 15) / 16 * 16);
+  static constexpr int kOffRow = kOffTs + (int)((sizeof(TsCtrl) + 15) / 16 * 16);
+  static constexpr int kBytes = (kOffRow + (int)sizeof(RowSel) + 127) / 128 * 128;
 };
+static_assert(HsSmem::kOffTs % 16 == 0 && HsSmem::kOffRow % 16 == 0, "control blocks aligned");
 static_assert(kHsCap * 8 <= kSelBins * 4, "the candidates fit the histogram's space");
 
 __device__ __forceinline__ uint32_t dsmem_atom_add(uint32_t addr, uint32_t v) {
@@ -289,8 +292,8 @@ __global__ void __launch_bounds__(kHsThreads) topk_hist_select_kernel(const HsPa
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + HsSmem::kOffHist);
   uint32_t* pass_hist = reinterpret_cast<uint32_t*>(smem + HsSmem::kOffPass);
   MrCtrl<1, kHsThreads>* c = reinterpret_cast<MrCtrl<1, kHsThreads>*>(smem + HsSmem::kOffCtrl);
-  TsCtrl* tc = reinterpret_cast<TsCtrl*>(smem + HsSmem::kOffCtrl + sizeof(MrCtrl<1, kHsThreads>));
-  RowSel* rs = reinterpret_cast<RowSel*>(smem + HsSmem::kOffCtrl + sizeof(MrCtrl<1, kHsThreads>) + sizeof(TsCtrl));
+  TsCtrl* tc = reinterpret_cast<TsCtrl*>(smem + HsSmem::kOffTs);
+  RowSel* rs = reinterpret_cast<RowSel*>(smem + HsSmem::kOffRow);
   uint32_t* cand_raw = reinterpret_cast<uint32_t*>(smem + HsSmem::kOffCand);
   uint32_t* cand_pos = cand_raw + kHsCap;
   const int tid = (int)threadIdx.x, lane = tid & 31;

@@ -45,8 +45,8 @@
 namespace dstopk {
 
 constexpr int kTsThreads = 1024;
-constexpr int kTsStages = 4;            // cp.async ring stages
-constexpr int kTsStageWords = 2048;     // 16-byte words per stage: a 128 KiB ring
+constexpr int kTsStages = 3;            // cp.async ring stages
+constexpr int kTsStageWords = 3072;     // 16-byte words per stage: a 144 KiB ring
 constexpr int kTsSample = 4096;         // sampled scores per CTA
 constexpr int kTsPosBits = 24;          // positions are below 2^24
 constexpr int kTsCap = 4096;            // stash entries per CTA (k <= 2048)
@@ -76,6 +76,7 @@ struct TsCtrl {
   uint32_t part[32][kTsMaxCluster];  // per-warp partial counts
   uint32_t above_of[kTsMaxCluster];
   uint32_t tval[16];        // every CTA: each CTA's stash threshold
+  uint32_t cutk, cutp;      // leader: the cut inside the k-th key's bin
 };
 
 // Shared memory, in order: histogram u32[4096] (the stash's offsets above the
@@ -91,6 +92,8 @@ __host__ __device__ constexpr int ts_off_ring(int C) { return ts_off_stash(C) + 
 __host__ __device__ constexpr int ts_ring_bytes() { return kTsStages * kTsStageWords * 16; }
 __host__ __device__ constexpr int ts_smem_bytes(int C) { return ts_off_ring(C) + ts_ring_bytes(); }
 static_assert(sizeof(TsCtrl) <= 1024, "control block");
+static_assert(ts_off_ctrl(1) % 16 == 0 && ts_off_stash(1) % 16 == 0 && ts_off_ring(1) % 16 == 0,
+              "the control block, the stash and the ring start on 16-byte boundaries");
 static_assert(ts_smem_bytes(kTsMaxCluster) <= 227 * 1024, "shared memory");
 static_assert((kTsMaxCluster - 1) * kTsCap * 8 <= ts_ring_bytes(), "received stashes fit the ring");
 
@@ -145,13 +148,33 @@ __device__ __forceinline__ uint32_t ts_find_bin(const uint32_t* h, int nb, uint3
   } else {
     for (int r = r0; r < r1; ++r) s += h[nb - 1 - r];
   }
-  if (threadIdx.x == 0) {
+  // two barriers: the warp totals out; every warp scans all of them itself
+  static_assert(NT % 32 == 0 && NT / 32 <= 32, "one warp's lanes cover the warp totals");
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) ctrl->wtot[warp] = incl;
+  __syncthreads();
+  const uint32_t wt = lane < NW ? ctrl->wtot[lane] : 0u;
+  uint32_t wi = wt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, wi, o);
+    if (lane >= o) wi += t;
+  }
+  const uint32_t wex = __shfl_sync(0xFFFFFFFFu, wi - wt, warp);
+  const uint32_t total = __shfl_sync(0xFFFFFFFFu, wi, 31);
+  const uint32_t excl = wex + incl - s;
+  if (threadIdx.x == 0 && (krem == 0u || krem > total)) {  // no such bin
     ctrl->bcast[0] = 0u;
     ctrl->bcast[1] = 0u;
     ctrl->bcast[2] = 0u;
   }
-  uint32_t total;
-  const uint32_t excl = ts_block_scan<NT>(s, ctrl, total);
   if (excl < krem && krem <= excl + s) {
     uint32_t acc = excl;
     for (int r = r0; r < r1; ++r) {
@@ -279,19 +302,6 @@ __device__ __forceinline__ void ts_block_minmax(uint32_t lo, uint32_t hi, TsCtrl
   gmax = ctrl->bcast[1];
 }
 
-// One slot of *counter to each lane of a warp that asks (all 32 lanes call
-// it): a ballot, one atomic, a population count.
-__device__ __forceinline__ uint32_t ts_warp_alloc1(bool take, uint32_t* counter) {
-  const int lane = threadIdx.x & 31;
-  const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
-  uint32_t base = 0u;
-  if (m != 0u) {
-    if (lane == 0) base = atomicAdd(counter, (uint32_t)__popc(m));
-    base = __shfl_sync(0xFFFFFFFFu, base, 0);
-  }
-  return base + (uint32_t)__popc(m & ((1u << lane) - 1u));
-}
-
 // Hands out n consecutive slots of *counter to each lane of a warp (all 32
 // lanes call it); returns this lane's first slot.
 __device__ __forceinline__ uint32_t ts_warp_alloc(uint32_t n, uint32_t* counter) {
@@ -403,9 +413,10 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   if (tid == 0) {
     ctrl->cnt = 0u;
     ctrl->out = 0u;
+    ctrl->bcast[3] = 0u;
   }
-  // the histogram of the stashed keys' offsets above t, counted after the
-  // stream (zeroed before the first barrier below)
+  // the leader's histogram of the stash's offsets above the threshold
+  // (zeroed before the first barrier below)
   constexpr int kRel = K::kBits == 32 ? 12 : 0;
   for (int i = tid; i < 4096; i += NT) hist[i] = 0u;
 
@@ -431,7 +442,10 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   if (pe >= 0) praw = (uint32_t)grow[pe];
 
   // ---- the cp.async ring: a thread copies V words per stage and later
-  // processes exactly those words, so the ring needs no block barrier
+  // processes exactly those words, so the ring needs no block barrier.  (A
+  // ring of bulk copies, one thread issuing each stage, streamed slower: a
+  // copy-only read of these rows takes 8.4 us with 16-byte loads from every
+  // thread and 9.7 us through a bulk-copy ring.)
   const int nst = (nfull + stage_words - 1) / stage_words;
   auto issue = [&](int st) {
     if (st < nst) {
@@ -572,20 +586,8 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   }
   __syncthreads();
 
-  // the offset histogram of the stash's keys >= t (a complete stash only)
-  {
-    const uint32_t n = ctrl->cnt;
-    if (n <= (uint32_t)kTsCap) {
-      for (int i = tid; i < (int)n; i += NT) {
-        const uint32_t key = K::key(st_raw[i]);
-        if (key >= t) atomicAdd(hist + min(4095u, (key - t) >> kRel), 1u);
-      }
-    }
-  }
-
-  // ---- in a cluster, every stash and histogram goes to the leader: stash c
-  // into the leader's ring (free once every CTA has streamed) at (c - 1) stash
-  // sizes, histogram c into its slot c
+  // ---- in a cluster, every stash goes to the leader: stash c into the
+  // leader's ring (free once every CTA has streamed) at (c - 1) stash sizes
   auto region = [&](int c) -> uint32_t* {
     return c == 0 ? st_raw : reinterpret_cast<uint32_t*>(ring + (size_t)(c - 1) * kTsCap * 8);
   };
@@ -606,38 +608,21 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   uint32_t cnt = ctrl->cnt;
   const bool ok = (counted || cnt >= (uint32_t)need) && cnt <= (uint32_t)kTsCap;
   bool all_ok = ok;
-  // The offset histograms meet in one frame: tmax, the largest of the CTAs'
-  // thresholds.  With every stash complete, the row's k-th key is >= each
-  // threshold of a slice that holds k keys (and slices that hold fewer have
-  // t = 0), so every key at or above the k-th is >= tmax and in a stash.
-  // CTA c's bin i is bin i - dc of that frame (dc = (tmax - t_c) >> kRel);
-  // its bins below dc drop out and its last bin stays the last.
-  uint32_t tmax = t, dmax = 0u;
-  uint32_t* acc = hist;  // the leader's merged histogram
+  // tmax, the largest of the CTAs' thresholds: with every stash complete, the
+  // row's k-th key is >= the threshold of each slice that holds k keys (and
+  // slices that hold fewer have t = 0), so every key at or above the k-th is
+  // >= tmax and in a stash
+  uint32_t tmax = t;
   if (C > 1) {
-    acc = shist;  // the ring's last stage: free after the stream, clear of the received stashes
-    if (crank == 0)
-      for (int i = tid; i < 4096; i += NT) acc[i] = 0u;
     if (tid < C) dsmem_st_u32(dsmem_map(smem_u32(&ctrl->tval[crank]), (uint32_t)tid), t);
     cluster_sync();  // every CTA has streamed: the leader's ring is free
-    for (int c = 0; c < C; ++c) tmax = max(tmax, ctrl->tval[c]);
-    for (int c = 0; c < C; ++c) dmax = max(dmax, (tmax - ctrl->tval[c]) >> kRel);
-    if (ok) {
-      const uint32_t dc = (tmax - t) >> kRel;
-      const uint32_t la = dsmem_map(smem_u32(acc), 0);
-      for (int i = tid; i < 4096; i += NT) {
-        const uint32_t h = hist[i];
-        if (h && (uint32_t)i >= dc) {
-          const uint32_t j = i == 4095 ? 4095u : (uint32_t)i - dc;
-          if (crank == 0) atomicAdd(acc + j, h);
-          else dsmem_red_add_u32(la + 4u * j, h);
-        }
-      }
-    }
     if (ok && crank != 0) ship(cnt);
     if (tid < C) dsmem_st_u32(dsmem_map(smem_u32(&ctrl->ok[crank]), (uint32_t)tid), ok ? 1u : 0u);
     cluster_sync();
-    for (int c = 0; c < C; ++c) all_ok &= ctrl->ok[c] != 0u;
+    for (int c = 0; c < C; ++c) {
+      all_ok &= ctrl->ok[c] != 0u;
+      tmax = max(tmax, ctrl->tval[c]);
+    }
   }
   if (tid == 0 && crank == 0) ctrl->tab[0] = cnt;
   // every CTA of the row has read the row's counts: the leader clears them
@@ -707,25 +692,79 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
       if (i < nc) f(K::key(rr[i]), rp[i]);
     }
   };
-  // With every stash as streamed, the offset histogram counts exactly the
-  // stash's keys >= t: the bin fb of the k-th key, and only that bin to
-  // resolve (mode 1: all of it is taken; mode 2: a cut inside it).
+  // The stash's keys >= tmax, counted in 4096 bins of their offset above
+  // tmax (2^12 float32 keys or one bfloat16 key per bin, the last bin taking
+  // everything above), place the k-th key: only its bin fb is resolved
+  // (mode 1: all of the bin is taken; mode 2: a cut inside it, from a warp
+  // sort of the bin's entries when they are few).
   int mode = 0;
   uint32_t fb = 0u;
   TsCut cut = TsCut{0u, 0, 0u};
   if (all_ok) {
+    visit_stash([&](uint32_t key, uint32_t) {
+      if (key >= tmax) atomicAdd(hist + min(4095u, (key - tmax) >> kRel), 1u);
+    });
+    __syncthreads();
     uint32_t above, inbin;
-    const uint32_t b = ts_find_bin<NT>(acc, 4096, (uint32_t)kk, ctrl, above, inbin);
-    // (bins 4095 - dc .. 4094 lack CTA c's keys counted in its last bin, so
-    // only a bin below all of them is exact)
-    if (b + dmax < 4095u && above < (uint32_t)kk && above + inbin >= (uint32_t)kk) {
+    const uint32_t b = ts_find_bin<NT>(hist, 4096, (uint32_t)kk, ctrl, above, inbin);
+    if (b < 4095u && above < (uint32_t)kk && above + inbin >= (uint32_t)kk) {
       fb = b;
       const int krem = kk - (int)above;
       if (inbin == (uint32_t)krem) {
         mode = 1;
       } else {
         mode = 2;
-        cut = ts_select<K, NT>(visit_stash, krem, hist, ctrl, (tmax >> kRel) + b, kRel);
+        // the bin's entries, listed in the ring's last stage (clear of the
+        // received stashes): inbin of them
+        constexpr int kListCap = 2048;
+        uint32_t* lk = shist;
+        uint32_t* lp = shist + kListCap;
+        visit_stash([&](uint32_t key, uint32_t pos) {
+          if (key >= tmax && min(4095u, (key - tmax) >> kRel) == b) {
+            const uint32_t s = atomicAdd(&ctrl->bcast[3], 1u);
+            if (s < (uint32_t)kListCap) {
+              lk[s] = key;
+              lp[s] = pos;
+            }
+          }
+        });
+        __syncthreads();
+        if (inbin <= 32u) {
+          if (tid < 32) {
+            // bitonic sort of the (at most 32) entries, greatest first: larger
+            // key, then lower position; lane krem - 1 holds the cut
+            uint32_t key = tid < (int)inbin ? lk[tid] : 0u;
+            uint32_t pos = tid < (int)inbin ? lp[tid] : 0xFFFFFFFFu;
+#pragma unroll
+            for (int w = 2; w <= 32; w <<= 1) {
+#pragma unroll
+              for (int j = w >> 1; j > 0; j >>= 1) {
+                const uint32_t ok2 = __shfl_xor_sync(0xFFFFFFFFu, key, j);
+                const uint32_t op2 = __shfl_xor_sync(0xFFFFFFFFu, pos, j);
+                const bool other_greater = ok2 > key || (ok2 == key && op2 < pos);
+                const bool keep_greater = ((tid & j) == 0) == ((tid & w) == 0);
+                if (other_greater == keep_greater) {
+                  key = ok2;
+                  pos = op2;
+                }
+              }
+            }
+            if (tid == krem - 1) {
+              ctrl->cutk = key;
+              ctrl->cutp = pos;
+            }
+          }
+          __syncthreads();
+          cut = TsCut{ctrl->cutk, 0, ctrl->cutp};
+        } else if (inbin <= (uint32_t)kListCap) {
+          const int nl = (int)inbin;
+          auto visit_list = [&](auto&& f) {
+            for (int i = tid; i < nl; i += NT) f(lk[i], lp[i]);
+          };
+          cut = ts_select<K, NT>(visit_list, krem, hist, ctrl, (tmax >> kRel) + b, kRel);
+        } else {
+          cut = ts_select<K, NT>(visit_stash, krem, hist, ctrl, (tmax >> kRel) + b, kRel);
+        }
       }
     }
   }
@@ -752,10 +791,14 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
     return rel > fb || (rel == fb && (mode == 1 || ts_taken(cut, key, pos)));
   };
   // every selected entry (exactly kk): one warp-level slot allocation per
-  // visit; with sorted_index gathered in shared memory first
+  // visit (a ballot and one atomic); with sorted_index gathered in shared
+  // memory first.  (Slots from a counting visit and a prefix over the warps,
+  // without atomics, came out slower: the visit costs more than the atomics.)
   uint32_t* sel_pos = hist;
   uint32_t* sel_raw = hist + 2048;
   const bool sorted = p.sorted != 0;
+  const int lane = tid & 31;
+  const uint32_t lt = (1u << lane) - 1u;
   for (int c = 0; c < C; ++c) {
     const int nc = min((int)ctrl->tab[c], kTsCap);
     const uint32_t* rr = region(c);
@@ -769,7 +812,13 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
         pos = rp[i];
         take = taken(K::key(raw), pos);
       }
-      const uint32_t slot = ts_warp_alloc1(take, &ctrl->out);
+      const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
+      uint32_t wb = 0u;
+      if (m != 0u) {
+        if (lane == 0) wb = atomicAdd(&ctrl->out, (uint32_t)__popc(m));
+        wb = __shfl_sync(0xFFFFFFFFu, wb, 0);
+      }
+      const uint32_t slot = wb + (uint32_t)__popc(m & lt);
       if (take && slot < (uint32_t)kk) {
         if (sorted) {
           sel_pos[slot] = pos;
