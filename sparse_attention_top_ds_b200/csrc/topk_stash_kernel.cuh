@@ -90,11 +90,15 @@ __host__ __device__ constexpr int ts_off_ctrl(int) { return 4096 * 4; }
 __host__ __device__ constexpr int ts_off_stash(int C) { return ts_off_ctrl(C) + 1024; }
 __host__ __device__ constexpr int ts_off_ring(int C) { return ts_off_stash(C) + kTsCap * 8; }
 __host__ __device__ constexpr int ts_ring_bytes() { return kTsStages * kTsStageWords * 16; }
-__host__ __device__ constexpr int ts_smem_bytes(int C) { return ts_off_ring(C) + ts_ring_bytes(); }
+// A pair (C = 2) receives the partner's stash in an area of its own after the
+// ring, so the partner can send it as soon as it has streamed.
+__host__ __device__ constexpr int ts_smem_bytes(int C) {
+  return ts_off_ring(C) + ts_ring_bytes() + (C == 2 ? kTsCap * 8 : 0);
+}
 static_assert(sizeof(TsCtrl) <= 1024, "control block");
 static_assert(ts_off_ctrl(1) % 16 == 0 && ts_off_stash(1) % 16 == 0 && ts_off_ring(1) % 16 == 0,
               "the control block, the stash and the ring start on 16-byte boundaries");
-static_assert(ts_smem_bytes(kTsMaxCluster) <= 227 * 1024, "shared memory");
+static_assert(ts_smem_bytes(kTsMaxCluster) <= 227 * 1024 && ts_smem_bytes(2) <= 227 * 1024, "shared memory");
 static_assert((kTsMaxCluster - 1) * kTsCap * 8 <= ts_ring_bytes(), "received stashes fit the ring");
 
 // Exclusive block-wide scan of one value per thread (every thread calls it):
@@ -370,6 +374,9 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   uint32_t* shist = reinterpret_cast<uint32_t*>(ring + (size_t)(kTsStages - 1) * stage_words * 16);
 
   const int row = (int)(blockIdx.x / csize);
+  // (arrive now, wait before the first access to another CTA's shared
+  // memory: by then every CTA of the cluster is running)
+  if (C > 1) cluster_arrive_relaxed();
   pdl_wait();
   pdl_launch_dependents();
   int L = p.n;
@@ -586,10 +593,14 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   }
   __syncthreads();
 
-  // ---- in a cluster, every stash goes to the leader: stash c into the
-  // leader's ring (free once every CTA has streamed) at (c - 1) stash sizes
+  // ---- in a cluster, every stash goes to the leader: a pair's partner into
+  // the leader's receive area, as soon as it has streamed; with four CTAs,
+  // stash c into the leader's ring (free once every CTA has streamed) at
+  // (c - 1) stash sizes
+  uint32_t* recv = reinterpret_cast<uint32_t*>(ring + ts_ring_bytes());
   auto region = [&](int c) -> uint32_t* {
-    return c == 0 ? st_raw : reinterpret_cast<uint32_t*>(ring + (size_t)(c - 1) * kTsCap * 8);
+    if (c == 0) return st_raw;
+    return C == 2 ? recv : reinterpret_cast<uint32_t*>(ring + (size_t)(c - 1) * kTsCap * 8);
   };
   auto ship = [&](uint32_t n) {
     const uint32_t nv = (n + 3u) >> 2;
@@ -614,11 +625,22 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   // >= tmax and in a stash
   uint32_t tmax = t;
   if (C > 1) {
-    if (tid < C) dsmem_st_u32(dsmem_map(smem_u32(&ctrl->tval[crank]), (uint32_t)tid), t);
-    cluster_sync();  // every CTA has streamed: the leader's ring is free
-    if (ok && crank != 0) ship(cnt);
-    if (tid < C) dsmem_st_u32(dsmem_map(smem_u32(&ctrl->ok[crank]), (uint32_t)tid), ok ? 1u : 0u);
-    cluster_sync();
+    cluster_wait();  // (the arrival at the start) every CTA of the cluster is running
+    if (C == 2) {
+      // one cluster barrier: the partner's stash, thresholds and verdicts in
+      if (ok && crank != 0) ship(cnt);
+      if (tid < C) {
+        dsmem_st_u32(dsmem_map(smem_u32(&ctrl->tval[crank]), (uint32_t)tid), t);
+        dsmem_st_u32(dsmem_map(smem_u32(&ctrl->ok[crank]), (uint32_t)tid), ok ? 1u : 0u);
+      }
+      cluster_sync();
+    } else {
+      if (tid < C) dsmem_st_u32(dsmem_map(smem_u32(&ctrl->tval[crank]), (uint32_t)tid), t);
+      cluster_sync();  // every CTA has streamed: the leader's ring is free
+      if (ok && crank != 0) ship(cnt);
+      if (tid < C) dsmem_st_u32(dsmem_map(smem_u32(&ctrl->ok[crank]), (uint32_t)tid), ok ? 1u : 0u);
+      cluster_sync();
+    }
     for (int c = 0; c < C; ++c) {
       all_ok &= ctrl->ok[c] != 0u;
       tmax = max(tmax, ctrl->tval[c]);
