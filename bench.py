@@ -384,7 +384,29 @@ ONLY_WORKLOADS = {
     "sampling": "top-k of 64 x 129280 float32 sampling rows, k = 1024, values and indices",
     "indexer-rows": "top-k of 64 x 131072 bfloat16 indexer-style rows, k = 2048, indices only",
     "prefill": "prefill indexer + top-k: 4096 rows x 64 heads x 128 bf16 vs 32768 keys, causal valid_len, k = 2048",
+    "floor": "read-only passes over the sampling rows (64 x 129280 float32, 8 copies rotating): 64, 128 and 256 "
+             "CTAs of 1024 threads",
+    "stash-phases": "phase stamps of the stash top-k kernel (needs DS_TOPK_LIB = libdstopk_debug.so): one call "
+                    "each of the sampling workload at k = 1024 and 64 and of 64 x 131072 bfloat16 rows at k = 2048",
 }
+
+STAMP_NAMES = ("start", "prologue", "sample counted", "threshold", "streamed", "merged", "leader: stash counted",
+               "leader: bin of the k-th key", "leader: bin resolved", "leader: emission written")
+
+
+def stamp_table(st):
+    """Median over CTAs of each phase stamp, µs after the first CTA's start."""
+    st = st.astype(np.float64)
+    used = st[:, 0] > 0
+    st = st[used]
+    t0 = st[:, 0].min()
+    out = {}
+    for j, nm in enumerate(STAMP_NAMES):
+        col = st[:, j]
+        col = col[col > 0]
+        if len(col):
+            out[nm] = round(float(np.median(col - t0)) / 1000.0, 2)
+    return {"ctas": int(used.sum()), "median_us_after_start": out}
 
 
 def run_only(args):
@@ -418,6 +440,36 @@ def run_only(args):
             oi = torch.empty((q.shape[0], k), dtype=torch.int32, device=dev)
             osc = torch.empty((q.shape[0], k), dtype=torch.float32, device=dev)
             fn = lambda: ds.ds_indexer_topk(qd, kd, wd, k, valid_len=vd, return_score=True, out_idx=oi, out_score=osc)
+        elif args.only == "floor":
+            x = torch.from_numpy(inputs.sampling(seed=inputs.SEED_SAMPLING + rank)[0]).to(dev)
+            xs = [x.clone() for _ in range(8)]
+            res = {}
+            for ctas in (64, 128, 256):
+                us = graph_times_us(lambda i: ds.ds_read_floor(xs[i % 8], ctas), 40, reps=5)
+                res[f"{ctas}_ctas"] = {"us_per_call": spread(us),
+                                       "gbs": round(x.numel() * 4 / (statistics.median(us) * 1e-6) / 1e9, 1)}
+            if rank == 0:
+                print(json.dumps({"floor": {"workload": ONLY_WORKLOADS["floor"], **res}}), flush=True)
+            return
+        elif args.only == "stash-phases":
+            if not ds.ds_debug_build():
+                raise RuntimeError("--only stash-phases needs DS_TOPK_LIB pointing at libdstopk_debug.so")
+            res = {}
+            samp = torch.from_numpy(inputs.sampling(seed=inputs.SEED_SAMPLING + rank)[0]).to(dev)
+            q, kc, w = inputs.indexer_factors(seed=inputs.SEED_INDEXER + rank, batch=64, n=131072)
+            rows = ds.ds_indexer_score(to(q), to(kc), torch.from_numpy(w).to(dev)).to(torch.bfloat16)
+            for name, xx, k in (("sampling_k1024", samp, 1024), ("sampling_k64", samp, 64),
+                                ("bf16_64x131072_k2048", rows, 2048)):
+                for _ in range(3):
+                    ds.ds_topk(xx, k, return_value=True)
+                torch.cuda.synchronize()
+                ds.ds_debug_stash_stamps(1024)  # clears
+                ds.ds_topk(xx, k, return_value=True)
+                torch.cuda.synchronize()
+                res[name] = stamp_table(ds.ds_debug_stash_stamps(1024))
+            if rank == 0:
+                print(json.dumps({"stash_phases": {"workload": ONLY_WORKLOADS["stash-phases"], **res}}), flush=True)
+            return
         elif args.only == "sampling":
             x = torch.from_numpy(inputs.sampling(seed=inputs.SEED_SAMPLING + rank)[0]).to(dev)
             oi = torch.empty((x.shape[0], 1024), dtype=torch.int32, device=dev)
@@ -804,6 +856,10 @@ def run_ours(args):
     if status != ds.DS_OK:
         raise RuntimeError(f"device status after prefill: {ds.strerror(status)}")
 
+    # the floor under the top-k: a read-only pass over the same rows, launched
+    # the same way (2 CTAs of 1024 threads per row), rotating the same copies
+    floor_us = graph_times_us(lambda i: ds.ds_read_floor(xs[i % R], 2 * B), R, reps=5)
+    (floor_med,) = max_over_ranks([statistics.median(floor_us)], dev)
     configs = measure_configs(ds, inputs, dev, rank, hbm_gbs, tflops)
     attention = measure_attention(ds, inputs, dev, stream, rank, hbm_gbs, tflops, ATTN_CALLS)
     qproj = measure_qproj(ds, inputs, dev, stream, rank, hbm_gbs, ATTN_CALLS)
@@ -867,6 +923,9 @@ def run_ours(args):
             "topk_pct_of_nominal_8tbs": round(100 * per_launch_gbs / NOMINAL_HBM_GBS, 1),
             "topk_rows_per_s": round(2 * B / ((t_k1 + t_k2) * 1e-3), 1),
             "topk_us_per_call": {"k1024": round(t_k1 * 1e3, 2), "k64": round(t_k2 * 1e3, 2)},
+            "topk_read_floor_us": {"us_per_call": round(floor_med, 2), "replays": spread(floor_us),
+                                   "what": "a kernel that only reads the same 33.1 MB of rows, 128 CTAs x 1024 "
+                                           "threads, 16-byte loads (ds_read_floor)"},
             "decode_us_per_step": round(t_dec * 1e3, 2),
             "decode_roofline_us": round(dec_roof_us, 3),
             "decode_frac_of_roofline": round(dec_roof_us / (t_dec * 1e3), 3),

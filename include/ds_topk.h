@@ -362,8 +362,30 @@ int ds_set_wait_limit(int64_t ns);
 int ds_plant_wait_fault(int launches);
 
 /* ds_debug_build -- 1 in libdstopk_debug.so (compiled with DS_DEBUG: device
- * range checks that record DS_ERR_RANGE), 0 in libdstopk.so. */
+ * range checks that record DS_ERR_RANGE, and phase stamps), 0 in libdstopk.so. */
 int ds_debug_build(void);
+
+/*
+ * ds_debug_stash_stamps -- libdstopk_debug.so only: the %globaltimer stamps
+ * (ns) that thread 0 of each of the first `ctas` CTAs of the stash top-k
+ * kernel recorded at the end of its phases since the last read, as `ctas` rows
+ * of 10 uint64 into host_dst (0: phase not reached); the stamps are cleared.
+ * Slots: start, prologue, sample counted, threshold, streamed, merged; then,
+ * in a row's leader CTA only: stash counted, bin of the k-th key, bin
+ * resolved, emission written.  Synchronises the device.  1 <= ctas <= 1024,
+ * else DS_ERR_ARG; DS_ERR_UNSUPPORTED in libdstopk.so.
+ * (No counterpart on the pages: measurement.)
+ */
+int ds_debug_stash_stamps(uint64_t* host_dst, int ctas);
+
+/*
+ * ds_read_floor -- enqueue a kernel that only reads `bytes` bytes at p (device,
+ * 16-byte aligned, bytes a multiple of 16) with 16-byte loads, split evenly
+ * over `ctas` CTAs of 1024 threads (1 .. 65535): the floor that a one-pass
+ * kernel over the same bytes cannot beat.  DS_ERR_ARG on a bad argument.
+ * (No counterpart on the pages: measurement.)
+ */
+int ds_read_floor(const void* p, int64_t bytes, int ctas, void* stream);
 
 /* ds_strerror -- a static, human-readable name for a status code. */
 const char* ds_strerror(int code);

@@ -20,6 +20,6 @@ from ._native import (  # noqa: F401
     DS_ERR_NOMEM, DS_ERR_RANGE, DS_MAX_K, DS_INDEXER_DIM, DS_INDEXER_MAX_HEADS, DS_ATTN_MAX_DIM, DS_ATTN_MAX_WINDOW,
     DS_ATTN_MAX_HEADS, DsError,
     ds_topk, ds_indexer_score, ds_indexer_topk, ds_indexer_topk_noalloc, ds_indexer_topk_ex, ds_indexer_qproj, ds_compress_fold, ds_sparse_attention, ds_get_device_status,
-    ds_release, ds_set_wait_limit, ds_plant_wait_fault, ds_debug_build,
+    ds_release, ds_set_wait_limit, ds_plant_wait_fault, ds_debug_build, ds_debug_stash_stamps, ds_read_floor,
     strerror, load, lib_path, DEBUG_LIB_PATH,
 )

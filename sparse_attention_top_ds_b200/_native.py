@@ -84,6 +84,10 @@ def load():
     lib.ds_plant_wait_fault.restype = i32
     lib.ds_debug_build.argtypes = []
     lib.ds_debug_build.restype = i32
+    lib.ds_debug_stash_stamps.argtypes = [vp, i32]
+    lib.ds_debug_stash_stamps.restype = i32
+    lib.ds_read_floor.argtypes = [vp, ctypes.c_int64, i32, vp]
+    lib.ds_read_floor.restype = i32
     _lib = lib
     return lib
 
@@ -150,6 +154,20 @@ def ds_plant_wait_fault(launches):
 def ds_debug_build():
     """True for the DS_DEBUG build (device range checks -> DS_ERR_RANGE)."""
     return bool(load().ds_debug_build())
+
+
+def ds_debug_stash_stamps(ctas):
+    """DS_DEBUG build: the stash top-k kernel's phase stamps (ns), [ctas, 10] uint64."""
+    import numpy as np
+    out = np.zeros((ctas, 10), dtype=np.uint64)
+    _check(load().ds_debug_stash_stamps(ctypes.c_void_p(out.ctypes.data), int(ctas)), "ds_debug_stash_stamps")
+    return out
+
+
+def ds_read_floor(x, ctas, stream=None):
+    """Enqueue a read-only pass over the CUDA tensor x (its bytes split over ctas CTAs)."""
+    _check(load().ds_read_floor(_ptr(x), x.numel() * x.element_size(), int(ctas), _stream_ptr(stream)),
+           "ds_read_floor")
 
 
 # ------------------------------------------------------------------ torch-tensor front end

@@ -52,6 +52,22 @@ constexpr int kTsPosBits = 24;          // positions are below 2^24
 constexpr int kTsCap = 4096;            // stash entries per CTA (k <= 2048)
 constexpr int kTsMaxCluster = 4;
 
+// Phase stamps of the DS_DEBUG build: thread 0 of CTA b records %globaltimer
+// at the end of each phase in ts_stamps[b][i] (read out by
+// ds_debug_stash_stamps); the release build compiles them away.
+constexpr int kTsStampCtas = 1024, kTsStampSlots = 10;
+#ifdef DS_DEBUG
+__device__ unsigned long long ts_stamps[kTsStampCtas][kTsStampSlots];
+#define TS_STAMP(i)                                                                     \
+  do {                                                                                  \
+    if (threadIdx.x == 0 && blockIdx.x < (unsigned)kTsStampCtas) ts_stamps[blockIdx.x][i] = globaltimer_ns(); \
+  } while (0)
+#else
+#define TS_STAMP(i) \
+  do {              \
+  } while (0)
+#endif
+
 struct TsParams {
   const void* scores;
   uint32_t* ghist;   // float32 rows: [batch, 4096] exact key histograms, or null (cleared here after use)
@@ -373,6 +389,7 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   uint8_t* ring = smem + ts_off_ring(C);
   uint32_t* shist = reinterpret_cast<uint32_t*>(ring + (size_t)(kTsStages - 1) * stage_words * 16);
 
+  TS_STAMP(0);  // start
   const int row = (int)(blockIdx.x / csize);
   // (arrive now, wait before the first access to another CTA's shared
   // memory: by then every CTA of the cluster is running)
@@ -427,6 +444,7 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   constexpr int kRel = K::kBits == 32 ? 12 : 0;
   for (int i = tid; i < 4096; i += NT) hist[i] = 0u;
 
+  TS_STAMP(1);  // prologue
   // ---- a strided sample of the full words (64 evenly spaced runs of run_w
   // words) when the slice does not fit the stash whole
   constexpr int SW = kTsSample / K::kVec;
@@ -498,6 +516,7 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
       }
     }
     __syncthreads();
+    TS_STAMP(2);  // sample counted
     const int ns = sw * K::kVec;
     const float lam = (float)need * (float)ns / (float)m;
     const int rk = min(ns, (int)ceilf(lam + 4.0f * sqrtf(lam) + 8.0f));
@@ -534,6 +553,7 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   // its stash slots with one atomic per stage.  The test is a float compare
   // against bound(t) (exact, or a superset that the stash's checks catch); the
   // per-element hit mask is built only by threads with a hit.
+  TS_STAMP(3);  // threshold
   const float tf = K::bound(t);
   for (int st = 0; st < nst; ++st) {
     issue(st + kTsStages - 1);
@@ -593,6 +613,7 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   }
   __syncthreads();
 
+  TS_STAMP(4);  // streamed
   // ---- in a cluster, every stash goes to the leader: a pair's partner into
   // the leader's receive area, as soon as it has streamed; with four CTAs,
   // stash c into the leader's ring (free once every CTA has streamed) at
@@ -628,6 +649,8 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
     cluster_wait();  // (the arrival at the start) every CTA of the cluster is running
     if (C == 2) {
       // one cluster barrier: the partner's stash, thresholds and verdicts in
+      // (writing the stash remotely during the stream instead slowed the
+      // stream more than it saved here)
       if (ok && crank != 0) ship(cnt);
       if (tid < C) {
         dsmem_st_u32(dsmem_map(smem_u32(&ctrl->tval[crank]), (uint32_t)tid), t);
@@ -696,6 +719,7 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
     if (C > 1) cluster_sync();
     else __syncthreads();
   }
+  TS_STAMP(5);  // merged (every CTA)
   if (crank != 0) return;
 
   // ---- the leader: the kk largest of the (merged) stash
@@ -727,8 +751,10 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
       if (key >= tmax) atomicAdd(hist + min(4095u, (key - tmax) >> kRel), 1u);
     });
     __syncthreads();
+    TS_STAMP(6);  // leader: stash counted
     uint32_t above, inbin;
     const uint32_t b = ts_find_bin<NT>(hist, 4096, (uint32_t)kk, ctrl, above, inbin);
+    TS_STAMP(7);  // leader: bin of the k-th key
     if (b < 4095u && above < (uint32_t)kk && above + inbin >= (uint32_t)kk) {
       fb = b;
       const int krem = kk - (int)above;
@@ -790,6 +816,7 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
       }
     }
   }
+  TS_STAMP(8);  // leader: the bin resolved (mode 1 or 2)
   if (mode == 0) {
     // the stash's keys share their top bits between its smallest and largest
     // key: the radix digits start below that common prefix, so the first pass
@@ -852,6 +879,7 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
       }
     }
   }
+  TS_STAMP(9);  // leader: thread 0's part of the emission written
   if (!sorted) return;
   __syncthreads();
   // ascending positions: bitonic sort of (position, score) pairs

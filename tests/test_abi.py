@@ -87,6 +87,22 @@ def test_wait_limit_and_planted_fault_arguments_need_no_gpu(lib):
     assert lib.ds_plant_wait_fault(0) == 0
 
 
+def test_measurement_entry_points_need_no_gpu(lib, debug_lib):
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    lib.ds_read_floor.argtypes = [vp, i64, ctypes.c_int, vp]
+    assert lib.ds_read_floor(None, 1024, 8, None) == -1                  # null
+    assert lib.ds_read_floor(vp(0x100008), 1024, 8, None) == -1          # not 16-byte aligned
+    assert lib.ds_read_floor(vp(0x100000), 1000, 8, None) == -1          # not a multiple of 16
+    assert lib.ds_read_floor(vp(0x100000), 1024, 0, None) == -1          # no CTA
+    lib.ds_debug_stash_stamps.argtypes = [vp, ctypes.c_int]
+    buf = (ctypes.c_uint64 * 10)()
+    assert lib.ds_debug_stash_stamps(buf, 1) == -4                       # release build: unsupported
+    debug_lib.ds_debug_stash_stamps.argtypes = [vp, ctypes.c_int]
+    assert debug_lib.ds_debug_stash_stamps(None, 1) == -1
+    assert debug_lib.ds_debug_stash_stamps(buf, 0) == -1
+    assert debug_lib.ds_debug_stash_stamps(buf, 1025) == -1
+
+
 def test_strerror(lib):
     lib.ds_strerror.restype = ctypes.c_char_p
     assert lib.ds_strerror(0) == b"DS_OK"
