@@ -744,7 +744,8 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   // (mode 1: all of the bin is taken; mode 2: a cut inside it, from a warp
   // sort of the bin's entries when they are few).
   int mode = 0;
-  uint32_t fb = 0u;
+  uint32_t fb = 0u, above_f = 0u;
+  int krem_f = 0;
   TsCut cut = TsCut{0u, 0, 0u};
   if (all_ok) {
     visit_stash([&](uint32_t key, uint32_t) {
@@ -758,8 +759,12 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
     if (b < 4095u && above < (uint32_t)kk && above + inbin >= (uint32_t)kk) {
       fb = b;
       const int krem = kk - (int)above;
+      above_f = above;
+      krem_f = krem;
       if (inbin == (uint32_t)krem) {
         mode = 1;
+      } else if (inbin <= 32u) {
+        mode = 3;  // resolved during the emission (below)
       } else {
         mode = 2;
         // the bin's entries, listed in the ring's last stage (clear of the
@@ -848,6 +853,84 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   const bool sorted = p.sorted != 0;
   const int lane = tid & 31;
   const uint32_t lt = (1u << lane) - 1u;
+  auto emit = [&](uint32_t slot, uint32_t pos, uint32_t raw) {
+    if (sorted) {
+      sel_pos[slot] = pos;
+      sel_raw[slot] = raw;
+    } else {
+      out_idx[slot] = (int32_t)pos;
+      if (out_val) out_val[slot] = (Raw)raw;
+    }
+  };
+  if (mode == 3) {
+    // One visit: the keys above the bin go out (slots 0 .. above - 1) and the
+    // bin's entries (at most 32) are listed; then one warp sorts them
+    // (bitonic, larger key then lower position first) and writes the first
+    // krem of them at slots above .. kk - 1.
+    uint32_t* lk = shist;
+    uint32_t* lp = shist + 32;
+    uint32_t* lr = shist + 64;
+    for (int c = 0; c < C; ++c) {
+      const int nc = min((int)ctrl->tab[c], kTsCap);
+      const uint32_t* rr = region(c);
+      const uint32_t* rp = rr + kTsCap;
+      for (int base = 0; base < nc; base += NT) {
+        const int i = base + tid;
+        uint32_t raw = 0u, pos = 0u, key = 0u;
+        bool up = false, inb = false;
+        if (i < nc) {
+          raw = rr[i];
+          pos = rp[i];
+          key = K::key(raw);
+          if (key >= tmax) {
+            const uint32_t rel = min(4095u, (key - tmax) >> kRel);
+            up = rel > fb;
+            inb = rel == fb;
+          }
+        }
+        const uint32_t m = __ballot_sync(0xFFFFFFFFu, up);
+        uint32_t wb = 0u;
+        if (m != 0u) {
+          if (lane == 0) wb = atomicAdd(&ctrl->out, (uint32_t)__popc(m));
+          wb = __shfl_sync(0xFFFFFFFFu, wb, 0);
+        }
+        const uint32_t slot = wb + (uint32_t)__popc(m & lt);
+        if (up && slot < above_f) emit(slot, pos, raw);
+        if (inb) {
+          const uint32_t s = atomicAdd(&ctrl->bcast[3], 1u);
+          if (s < 32u) {
+            lk[s] = key;
+            lp[s] = pos;
+            lr[s] = raw;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    if (tid < 32) {
+      const int n = (int)min(ctrl->bcast[3], 32u);
+      uint32_t key = tid < n ? lk[tid] : 0u;
+      uint32_t pos = tid < n ? lp[tid] : 0xFFFFFFFFu;
+      uint32_t raw = tid < n ? lr[tid] : 0u;
+#pragma unroll
+      for (int w = 2; w <= 32; w <<= 1) {
+#pragma unroll
+        for (int j = w >> 1; j > 0; j >>= 1) {
+          const uint32_t ok2 = __shfl_xor_sync(0xFFFFFFFFu, key, j);
+          const uint32_t op2 = __shfl_xor_sync(0xFFFFFFFFu, pos, j);
+          const uint32_t or2 = __shfl_xor_sync(0xFFFFFFFFu, raw, j);
+          const bool other_greater = ok2 > key || (ok2 == key && op2 < pos);
+          const bool keep_greater = ((tid & j) == 0) == ((tid & w) == 0);
+          if (other_greater == keep_greater) {
+            key = ok2;
+            pos = op2;
+            raw = or2;
+          }
+        }
+      }
+      if (tid < krem_f) emit(above_f + (uint32_t)tid, pos, raw);
+    }
+  } else {
   for (int c = 0; c < C; ++c) {
     const int nc = min((int)ctrl->tab[c], kTsCap);
     const uint32_t* rr = region(c);
@@ -868,16 +951,9 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
         wb = __shfl_sync(0xFFFFFFFFu, wb, 0);
       }
       const uint32_t slot = wb + (uint32_t)__popc(m & lt);
-      if (take && slot < (uint32_t)kk) {
-        if (sorted) {
-          sel_pos[slot] = pos;
-          sel_raw[slot] = raw;
-        } else {
-          out_idx[slot] = (int32_t)pos;
-          if (out_val) out_val[slot] = (Raw)raw;
-        }
-      }
+      if (take && slot < (uint32_t)kk) emit(slot, pos, raw);
     }
+  }
   }
   TS_STAMP(9);  // leader: thread 0's part of the emission written
   if (!sorted) return;
