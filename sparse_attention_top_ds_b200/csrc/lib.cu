@@ -595,7 +595,12 @@ static int launch_score_hist(const void* q, const void* kc, const float* w, int 
 static int launch_hist_select(const float* scores, uint32_t* ghist, const int32_t* vl, int32_t* out_idx,
                               float* out_score, int B, int S, int k, int sorted, cudaStream_t st, DeviceState* s) {
   int C = 1;
-  while (2 * C <= g_max_cluster && (long)B * 2 * C <= s->num_sms && S / (2 * C) >= 1024) C *= 2;
+  int cmax = g_max_cluster;
+  if (const char* f = getenv("DS_HS_CLUSTER")) {  // tuning sweeps only: the largest cluster allowed
+    const int v = atoi(f);
+    if (v == 1 || v == 2 || v == 4 || v == 8 || v == 16) cmax = std::min(cmax, v);
+  }
+  while (2 * C <= cmax && (long)B * 2 * C <= s->num_sms && S / (2 * C) >= 1024) C *= 2;
   HsParams h;
   memset(&h, 0, sizeof(h));
   h.scores = scores;

@@ -53,15 +53,20 @@ struct MrCtrl {
 // For nr <= NR histograms of nb bins (bin b of row r read as get(r, b)), find
 // per row the bin b with #(keys in bins > b) < target(r) <= #(keys in bins >= b);
 // the results land in c->res[r] = {bin, above, inbin} ({0, 0, 0} when target
-// is 0).  Every thread calls it; three block barriers serve all rows.
+// is 0).  Every thread calls it; two block barriers serve all rows.
 template <int NTH, int NR, class Get, class Target>
 __device__ __forceinline__ void mr_find_bin(Get&& get, int nb, int nr, Target&& target, MrCtrl<NR, NTH>* c) {
-  static_assert(NTH % 32 == 0 && NTH / 32 <= 32 && NR <= NTH / 32, "one warp scans each row's warp totals");
+  static_assert(NTH % 32 == 0 && NTH / 32 <= 32 && NR <= NTH / 32, "one warp's lanes cover a row's warp totals");
   constexpr int NW = NTH / 32;
   const int tid = (int)threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bpt = (nb + NTH - 1) / NTH;
   const int r0 = tid * bpt;  // first rank owned (0 = the top bin)
   const int r1 = min(nb, r0 + bpt);
+  if (tid < nr) {
+    c->res[tid][0] = 0u;
+    c->res[tid][1] = 0u;
+    c->res[tid][2] = 0u;
+  }
 #pragma unroll 1
   for (int r = 0; r < nr; ++r) {
     uint32_t a = 0u;
@@ -77,26 +82,19 @@ __device__ __forceinline__ void mr_find_bin(Get&& get, int nb, int nr, Target&& 
     if (lane == 31) c->wtot[r][warp] = in;
   }
   __syncthreads();
-  if (warp < nr) {
-    const uint32_t x = lane < NW ? c->wtot[warp][lane] : 0u;
+  // two barriers in all: every warp scans a row's warp totals itself
+#pragma unroll 1
+  for (int r = 0; r < nr; ++r) {
+    const uint32_t x = lane < NW ? c->wtot[r][lane] : 0u;
     uint32_t y = x;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, y, o);
       if (lane >= o) y += t;
     }
-    if (lane < NW) c->wex[warp][lane] = y - x;
-    if (lane == 0) {
-      c->res[warp][0] = 0u;
-      c->res[warp][1] = 0u;
-      c->res[warp][2] = 0u;
-    }
-  }
-  __syncthreads();
-#pragma unroll 1
-  for (int r = 0; r < nr; ++r) {
+    const uint32_t wex = __shfl_sync(0xFFFFFFFFu, y - x, warp);
     const uint32_t tg = target(r), a = c->part[r][tid];
-    const uint32_t excl = c->wex[r][warp] + c->incl[r][tid] - a;
+    const uint32_t excl = wex + c->incl[r][tid] - a;
     if (excl < tg && tg <= excl + a) {
       uint32_t acc = excl;
       for (int i = r0; i < r1; ++i) {
