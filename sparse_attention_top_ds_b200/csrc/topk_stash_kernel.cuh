@@ -16,17 +16,20 @@
 //  * The k largest of a slice always contain that slice's share of the row's
 //    k largest, so a CTA only checks its own count: the stash must hold at
 //    least min(k, slice) keys and fit.  In a cluster every CTA then copies its
-//    stash into the leader CTA (distributed shared memory).
-//  * While it stashes, each CTA counts the stashed keys in a histogram of
-//    their offset above t (4096 bins of 2^12 float32 keys, or of single
-//    bfloat16 keys; the last bin takes everything above).  The leader adds
-//    the CTAs' histograms, finds the bin of the row's k-th key in it, and
-//    resolves only that bin: one radix pass over the stash's keys inside it
-//    (none for bfloat16), then positions for ties.  When the k-th key lies in
-//    the last bin (or a CTA's stash was redone, see below), the leader instead
-//    selects from the whole stash, one radix pass per digit below the
-//    common prefix of its smallest and largest key.
-//    Every selected entry is written out with one warp-level atomic per
+//    stash into the leader CTA (distributed shared memory): a pair's partner
+//    into a receive area of the leader's own as soon as it has streamed,
+//    behind one cluster barrier; four CTAs into the leader's ring, behind two.
+//  * The row's k-th key is at or above tmax, the largest of the CTAs'
+//    thresholds.  The leader counts the merged stash's keys >= tmax in 4096
+//    bins of their offset above tmax (2^12 float32 keys, or single bfloat16
+//    keys; the last bin takes everything above), finds the bin of the k-th
+//    key, and resolves only that bin: when it holds at most 32 entries, the
+//    emission visit lists them and one warp sorts them; otherwise a radix pass
+//    over a list of the bin's keys (none for bfloat16), then positions for
+//    ties.  When the k-th key lies in the last bin (or a CTA's stash was
+//    redone, see below), the leader instead selects from the whole stash, one
+//    radix pass per digit below the common prefix of its smallest and largest
+//    key.  Every selected entry is written out with one warp-level atomic per
 //    visit, and sorted_index sorts the selection by position first.
 //  * A CTA whose stash came out short or too long (an unlucky sample, many
 //    equal keys) re-reads its slice from L2 and finds its exact k-th (key,
