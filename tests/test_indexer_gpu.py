@@ -257,6 +257,26 @@ def test_fused_all_scores_equal(cuda_device, B, S, L):
     assert np.all(score.cpu().numpy()[1, :min(2048, L // 3)] == 0.0)
 
 
+@pytest.mark.parametrize("cluster", ["1", "2", "4", "8", "16"])
+def test_split_row_selection_every_cluster_size(cuda_device, cluster, monkeypatch):
+    # the split-row selection with its cluster capped (DS_HS_CLUSTER, a tuning
+    # knob): every size must give the oracle's selection, sorted or not
+    monkeypatch.setenv("DS_HS_CLUSTER", cluster)
+    q, kc, w, vl = inputs.decode(seed=57, batch=8, S=32768, vl_lo=4096, vl_hi=32768)
+    qd, kd, wd, vd = dev_inputs(q, kc, w, vl)
+    idx, score = ds.ds_indexer_topk(qd, kd, wd, 1024, valid_len=vd, return_score=True)
+    torch.cuda.synchronize()
+    assert ds.ds_get_device_status() == ds.DS_OK
+    check_selection(q, kc, w, vl, 1024, idx.cpu().numpy(), score.cpu().numpy())
+    sidx, _ = ds.ds_indexer_topk_ex(qd, kd, wd, 1024, valid_len=vd, sorted_index=True)
+    torch.cuda.synchronize()
+    si = sidx.cpu().numpy()
+    for t in range(8):
+        m = int((si[t] >= 0).sum())
+        assert np.all(np.diff(si[t, :m]) > 0), f"row {t}: not ascending"
+        assert np.array_equal(si[t, :m], np.sort(idx.cpu().numpy()[t, :m])), f"row {t}: sorted set differs"
+
+
 @pytest.mark.parametrize("B", [8, 600])
 def test_fused_graph_replay(cuda_device, B):
     # the split-row path leaves its histograms and tickets zero for the next
