@@ -356,7 +356,8 @@ int ds_set_wait_limit(int64_t ns);
  * limit.  The kernel then scores that CTA's remaining positions as -inf, lets
  * its copies in flight land, frees its tensor memory and returns; the call's
  * status is DS_ERR_TIMEOUT.  0 disarms.  launches >= 0, else DS_ERR_ARG.
- * Nothing traps, and the next call without the fault runs normally.
+ * Nothing traps, and the next call without the fault runs normally.  A
+ * launch captured into a CUDA graph keeps the fault it was captured with.
  * (No counterpart on the pages.)
  */
 int ds_plant_wait_fault(int launches);
