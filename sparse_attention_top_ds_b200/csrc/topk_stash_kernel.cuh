@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
   constexpr int kShift0 = K::kBits - 12;
   constexpr int stage_words = kTsStageWords;
   constexpr int V = stage_words / NT;  // words per thread per stage
-  static_assert(V * NT == stage_words && V * K::kVec <= 64, "ring stage");
+  static_assert(V * NT == stage_words && V * K::kVec <= 32, "ring stage: one hit bit per score in a word");
 
   const int tid = threadIdx.x;
   const uint32_t crank = cluster_ctarank();
@@ -554,8 +554,8 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
 
   // ---- one pass: every key >= t is stashed with its position; a warp takes
   // its stash slots with one atomic per stage.  The test is a float compare
-  // against bound(t) (exact, or a superset that the stash's checks catch); the
-  // per-element hit mask is built only by threads with a hit.
+  // against bound(t) (exact, or a superset that the stash's checks catch)
+  // into a 32-bit hit mask; only the set bits are then visited.
   TS_STAMP(3);  // threshold
   const float tf = K::bound(t);
   for (int st = 0; st < nst; ++st) {
@@ -563,7 +563,7 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
     asm volatile("cp.async.wait_group %0;" ::"n"(kTsStages - 1) : "memory");
     const int slot = st % kTsStages;
     uint4 x[V];
-    bool anyh = false;
+    uint32_t hits = 0u;  // one bit per score of this thread's words
 #pragma unroll
     for (int v = 0; v < V; ++v) {
       const int w = st * stage_words + v * NT + tid;
@@ -571,36 +571,31 @@ __global__ void __launch_bounds__(NT, 1) topk_stash_kernel(const TsParams p) {
       if (w < nfull) {
         x[v] = *reinterpret_cast<const uint4*>(ring + ((size_t)slot * stage_words + v * NT + tid) * 16);
 #pragma unroll
-        for (int j = 0; j < K::kVec; ++j) anyh |= K::ge(x[v], j, tf);
+        for (int j = 0; j < K::kVec; ++j) hits |= (uint32_t)K::ge(x[v], j, tf) << (v * K::kVec + j);
       }
     }
-    unsigned long long hits = 0ull;
-    if (anyh) {
+    uint32_t pos = ts_warp_alloc((uint32_t)__popc(hits), &ctrl->cnt);
+    // only the hits are visited (a warp runs as many rounds as its busiest lane)
+    while (hits) {
+      const int j = __ffs(hits) - 1;
+      hits &= hits - 1u;
+      const int v = j / K::kVec, e = j % K::kVec;
+      // the hit's 32-bit word (4 per 16-byte word), then its half for bfloat16
+      constexpr int kPerWord = K::kVec / 4;
+      const int wj = j / kPerWord;
+      uint32_t word = 0u;
 #pragma unroll
-      for (int v = 0; v < V; ++v) {
-        if (st * stage_words + v * NT + tid < nfull) {
-#pragma unroll
-          for (int j = 0; j < K::kVec; ++j)
-            hits |= (unsigned long long)K::ge(x[v], j, tf) << (v * K::kVec + j);
-        }
+      for (int q = 0; q < V * 4; ++q) {
+        const uint4& xv = x[q / 4];
+        const uint32_t c = (q & 3) == 0 ? xv.x : ((q & 3) == 1 ? xv.y : ((q & 3) == 2 ? xv.z : xv.w));
+        word = q == wj ? c : word;
       }
-    }
-    uint32_t pos = ts_warp_alloc((uint32_t)__popcll(hits), &ctrl->cnt);
-    if (hits) {
-#pragma unroll
-      for (int v = 0; v < V; ++v) {
-        const int e0 = e_f0 + (st * stage_words + v * NT + tid) * K::kVec;
-#pragma unroll
-        for (int j = 0; j < K::kVec; ++j) {
-          if ((hits >> (v * K::kVec + j)) & 1ull) {
-            if (pos < (uint32_t)kTsCap) {
-              st_raw[pos] = K::slot(x[v], j);
-              st_pos[pos] = (uint32_t)(e0 + j);
-            }
-            ++pos;
-          }
-        }
+      const uint32_t raw = kPerWord == 1 ? word : ((j & 1) ? (word >> 16) : (word & 0xFFFFu));
+      if (pos < (uint32_t)kTsCap) {
+        st_raw[pos] = raw;
+        st_pos[pos] = (uint32_t)(e_f0 + (st * stage_words + v * NT + tid) * K::kVec + e);
       }
+      ++pos;
     }
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
