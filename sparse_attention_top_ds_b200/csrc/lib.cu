@@ -168,8 +168,7 @@ static bool topk_cluster16_ok() {
   cudaFuncSetAttribute(topk_cluster_kernel<BF16Keys, 256>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   cudaFuncSetAttribute(topk_cluster_kernel<BF16Keys, 512>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   cudaFuncSetAttribute(topk_hist_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(16, 1, 1);
   cfg.blockDim = dim3(256, 1, 1);
   cfg.dynamicSmemBytes = (size_t)kTopkSmemBytes;
@@ -190,8 +189,7 @@ static bool topk_cluster16_ok() {
 
 template <class K, int NT>
 static cudaError_t launch_topk(const TopkParams& p, int C, cudaStream_t st) {
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(p.batch * C), 1, 1);
   cfg.blockDim = dim3(NT, 1, 1);
   cfg.dynamicSmemBytes = (size_t)kTopkSmemBytes;
@@ -238,8 +236,7 @@ static int topk_stash_enqueue(const void* scores, int batch, int n, int k, int d
   p.return_value = return_value ? 1 : 0;
   p.sorted = sorted_index ? 1 : 0;
   p.status = s->status;
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(batch * C), 1, 1);
   cfg.blockDim = dim3(kTsThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)ts_smem_bytes(C);
@@ -435,8 +432,7 @@ static int launch_score(const void* q, const void* kc, const float* w, int B, in
   p.key_per_row = per_row ? 1 : 0;
   p.wait_ns = wait_limit();
   p.fault = take_planted_fault();
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(groups * cpg), 1, 1);
   cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)Cfg::kSmemBytes;
@@ -576,8 +572,7 @@ static int launch_score_hist(const void* q, const void* kc, const float* w, int 
   p.ghist = ghist;
   p.wait_ns = wait_limit();
   p.fault = take_planted_fault();
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(((B + NT - 1) / NT) * cpg), 1, 1);
   cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)Cfg::kSmemBytes;
@@ -614,8 +609,7 @@ static int launch_hist_select(const float* scores, uint32_t* ghist, const int32_
   h.slice = ((S + C - 1) / C + 3) / 4 * 4;
   h.sorted = sorted;
   h.status = s->status;
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(B * C), 1, 1);
   cfg.blockDim = dim3(kHsThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)HsSmem::kBytes;
@@ -764,8 +758,7 @@ static int attention_enqueue(const uint16_t* q, const uint16_t* kv, long long kv
     if (NS > 0) {
       CUtensorMap tq;
       if (!encode_attn_q(q + (size_t)b0 * H * D, (long long)nb * H, D, &tq)) return DS_ERR_ARG;
-      cudaLaunchConfig_t cfg;
-      memset(&cfg, 0, sizeof(cfg));
+      cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3((unsigned)NS, (unsigned)HT, (unsigned)nb);
       cfg.blockDim = dim3(kAttnThreads, 1, 1);
       cfg.dynamicSmemBytes = (size_t)AttnSmem::bytes(D);
@@ -779,8 +772,7 @@ static int attention_enqueue(const uint16_t* q, const uint16_t* kv, long long kv
     const int G = (NS > 1 && 2L * (D / kPvSlice) * HT * nb <= s->num_sms) ? 2 : 1;
     const PvCfg* pc = pv_pick(NS);
     if (!pc) return DS_ERR_ARG;
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(D / kPvSlice), (unsigned)G, (unsigned)(HT * nb));
     cfg.blockDim = dim3(kPvWarps * 32, 1, 1);
     cfg.dynamicSmemBytes = (size_t)pc->bytes(NS);
@@ -844,8 +836,7 @@ static int qproj_tc_enqueue(const void* x, const void* wq, const void* ww, int T
   p.nblk = nblk;
   p.bpb = bpb;
   p.nqb = nqb;
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)nrb, (unsigned)G, (unsigned)ntg);
   cfg.blockDim = dim3(128, 1, 1);
   cfg.dynamicSmemBytes = (size_t)QtSmem::kBytes;
@@ -1125,8 +1116,7 @@ extern "C" int ds_indexer_qproj(const void* x, const void* wq, const void* ww, i
   p.nq = heads * d;
   p.nrows = p.nq + (ww ? heads : 0);
   const int ntasks = (p.nrows + kQpRows - 1) / kQpRows;
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)std::min((ntasks + 7) / 8, s->num_sms), (unsigned)((T + kQpTok - 1) / kQpTok), 1);
   cfg.blockDim = dim3(kQpThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)kQpTok * d_in * 2 + 8 * 32 * 33 * 4;
@@ -1172,8 +1162,7 @@ extern "C" int ds_compress_fold(const void* rows, int batch, int D, int64_t rows
   p.out_bstride = (long long)out_batch_stride;
   p.B = batch;
   p.D = D;
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((batch + kCfWarps - 1) / kCfWarps), 1, 1);
   cfg.blockDim = dim3(kCfWarps * 32, 1, 1);
   cfg.stream = static_cast<cudaStream_t>(stream);
