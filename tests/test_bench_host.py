@@ -1,6 +1,7 @@
 """Host-side logic of bench.py (CPU only): algorithmic byte / FLOP counts (top-k,
-decode step, sparse attention), the clock-log summary, and the max-over-ranks
-reduction with two gloo ranks."""
+decode step, sparse attention), the clock-log summary, the phase-stamp table,
+the replay spread and input rotation, and the max-over-ranks reduction with two
+gloo ranks."""
 
 import os
 import socket
@@ -86,3 +87,27 @@ def test_max_over_two_gloo_ranks():
     for r, ws, got in res:
         assert ws == 2
         assert got == [2.0, 10.0]
+
+
+def test_stamp_table_medians_after_the_first_start():
+    import numpy as np
+    # two CTAs that started 1000 ns apart; the second never reached the leader
+    # phases (0 = not reached); unused rows (start 0) are ignored
+    st = np.zeros((4, 10), dtype=np.uint64)
+    st[0, :6] = [5000, 6000, 7000, 8000, 9000, 10000]
+    st[0, 6:] = [11000, 12000, 13000, 14000]
+    st[1, :6] = [6000, 7000, 8000, 9000, 10000, 11000]
+    t = bench.stamp_table(st)
+    assert t["ctas"] == 2
+    m = t["median_us_after_start"]
+    assert m["start"] == 0.5 and m["prologue"] == 1.5 and m["merged"] == 5.5
+    assert m["leader: stash counted"] == 6.0 and m["leader: emission written"] == 9.0
+
+
+def test_spread_and_rotation():
+    s = bench.spread([3.0, 1.0, 2.0])
+    assert s == {"median": 2.0, "min": 1.0, "max": 3.0, "replays": 3}
+    # copies whose cycle reads more than 2x L2 between two uses of one copy
+    r = bench.rotation(33_095_680)
+    assert (r - 1) * 33_095_680 > 2 * bench.L2_BYTES
+    assert bench.rotation(1) == 4096  # capped
