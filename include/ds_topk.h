@@ -138,11 +138,13 @@ int ds_indexer_score(const void* q, const void* kcache, const float* w,
  *    rows 2 and 3, and "The top-k on the GPSIMD engine": the scores feed the
  *    top-k as they are produced.)
  *
- * When a row is scored by several CTAs (few rows, as in decode) the scorer
- * also counts every score in an exact per-row histogram of its key's top 12
- * bits, and the selection starts from the threshold bin those counts give;
- * with many rows the scores go to the scratch buffer and ds_topk's kernel
- * selects them.  The result is the same either way.
+ * The scorer writes the score rows to the scratch buffer and also counts
+ * every score in an exact per-row histogram of its key's top 12 bits; the
+ * selection starts from the threshold bin those counts give.  Rows scored by
+ * several CTAs (few rows, as in decode) are selected by a cluster per row
+ * that splits the row; rows scored whole by one CTA (many rows, as in
+ * prefill) by ds_topk's one-pass kernel, which then draws no sample.  The
+ * result is the same either way.
  *
  * q, kcache, w, batch, heads, d, S, valid_len  as for ds_indexer_score.
  * k          1 <= k <= DS_MAX_K.
