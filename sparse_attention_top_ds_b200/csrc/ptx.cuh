@@ -11,7 +11,6 @@ namespace dstopk {
 // Status codes written to the per-device status word (match include/ds_topk.h).
 constexpr int kErrCuda = -2;     // DS_ERR_CUDA: a launch found its set-up inconsistent
 constexpr int kErrTimeout = -3;  // DS_ERR_TIMEOUT
-constexpr int kErrInternal = kErrCuda;
 constexpr int kErrRange = -6;    // DS_ERR_RANGE (recorded by DS_DEBUG builds only)
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
@@ -113,34 +112,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       : "memory");
 }
 
-// Same, with an L2 eviction-priority hint (policy from createpolicy).
-__device__ __forceinline__ void bulk_g2s_hint(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
-                                              uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], "
-      "%4;" ::"r"(dst),
-      "l"(src), "r"(bytes), "r"(bar), "l"(policy)
-      : "memory");
-}
-
-// One contiguous shared -> global copy through the TMA unit (bulk-group
-// completion); `src`, `dst` and `bytes` multiples of 16.
-__device__ __forceinline__ void bulk_s2g(void* dst, uint32_t src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-
-// Wait until every bulk copy this thread committed has completed.
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
 // ------------------------------------------------------------------ clusters
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -180,12 +151,6 @@ __device__ __forceinline__ uint32_t dsmem_map(uint32_t local, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
   return r;
-}
-
-__device__ __forceinline__ uint32_t dsmem_ld_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
 }
 
 __device__ __forceinline__ void dsmem_red_add_u32(uint32_t addr, uint32_t v) {
